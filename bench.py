@@ -1,0 +1,362 @@
+"""Benchmark of the GR-KAN hot path on B200: one step = forward (y) + backward
+(dx, then dA / dB through the two-stage reduction) over one batch of
+synthetic KAT-shaped activations resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config kat_b]
+    python bench.py --impl reference ...      # the fp64 oracle on host cores
+
+Prints one JSON line (rank 0). For N > 1 launch with torchrun; every rank
+processes its own batch (weak scaling) and the per-rank float64 gradient sums
+are all-gathered over NCCL and merged in rank order.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from group_rational_kan_b200 import accounting  # noqa: E402
+
+METRIC = "GR-KAN fwd+bwd elements/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+UNIT = "elements/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="kat_b", choices=list(synth.WORKLOADS))
+    ap.add_argument("--ng", type=int, default=None, help="groups for the stress workload")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def dtype_name(w):
+    return "f32" if w.dtype == synth.F32 else "bf16"
+
+
+# --- clocks ---------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --- reference arm / CPU baseline: the fp64 oracle on host cores ----------------------
+
+def oracle_step(orc, w, x, dy, a, b):
+    orc.forward(x, a, b, w.n_g)
+    orc.backward_elem(x, dy, a, b, w.n_g)
+    orc.coef_grads(x, dy, a, b, w.n_g)
+
+
+def oracle_rate(w, target_s, min_rows=1):
+    """Time the oracle (as it stands) on the first rows of the workload."""
+    import oracle
+    orc = oracle.Oracle()
+    rows = max(min_rows, 1)
+    while True:
+        s = w.with_rows(rows)
+        x, dy = s.x(), s.dy()
+        a, b = s.coefficients()
+        t0 = time.perf_counter()
+        oracle_step(orc, s, x, dy, a, b)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or rows >= w.rows:
+            return rows, dt, orc.max_threads()
+        rows = min(w.rows, max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.05)))
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    orc = oracle.Oracle()
+    # size one step so that warmup + steps take about two minutes in all
+    budget = 120.0 / max(args.steps + args.warmup, 1)
+    rows, dt, cores = oracle_rate(w, min(budget, 2.0))
+    per_row = dt / rows
+    rows = max(1, min(w.rows, int(budget / per_row)))
+    s = w.with_rows(rows)
+    x, dy = s.x(), s.dy()
+    a, b = s.coefficients()
+    for _ in range(args.warmup):
+        oracle_step(orc, s, x, dy, a, b)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(orc, s, x, dy, a, b)
+    el = time.perf_counter() - t0
+    value = s.elems * args.steps / el
+    sample = "first %d of %d rows of %s per step (%d elements), fwd y + bwd dx + dA/dB" % (
+        rows, w.rows, w.name, s.elems)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(w.describe(), rows_per_step=rows),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+# --- our arm ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    w = synth.workload(args.config, n_g=args.ng)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import group_rational_kan_b200 as grk
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w.seed = rank  # weak scaling: every rank its own batch
+    B, N, d, n_g, m, n, dt = w.B, w.N, w.d, w.n_g, w.m, w.n, w.dtype
+    E = w.elems
+    es = w.es
+    tdt = torch.float32 if dt == synth.F32 else torch.bfloat16
+    nbytes = E * es
+
+    # inputs: generated on the host into pinned memory, then copied to HBM
+    x_h = torch.empty((B, N, d), dtype=tdt, pin_memory=True)
+    dy_h = torch.empty((B, N, d), dtype=tdt, pin_memory=True)
+    synth.fill_ptr(x_h.data_ptr(), E, dt, w.seed, synth.X_STREAM, w.x_kind, w.x_scale, w.x_clip)
+    synth.fill_ptr(dy_h.data_ptr(), E, dt, w.seed, synth.DY_STREAM, synth.KIND_NORMAL, w.dy_scale)
+    a_np, b_np = w.coefficients()
+    a = torch.from_numpy(a_np).to(dev)
+    b = torch.from_numpy(b_np).to(dev)
+    x = x_h.to(dev)
+    dy = dy_h.to(dev)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    dA = torch.empty((n_g, m + 1), dtype=torch.float32, device=dev)
+    dB = torch.empty((n_g, n), dtype=torch.float32, device=dev)
+    wsb = grk.grkan_backward_workspace_bytes(B, N, d, n_g, m, n, dt)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    K = m + 1 + n
+    sums64 = torch.empty((n_g, K), dtype=torch.float64, device=dev) if world > 1 else None
+    gathered = torch.empty((world, n_g, K), dtype=torch.float64, device=dev) if world > 1 else None
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    path_f = grk.grkan_forward_path(x, y, B, N, d, n_g, m, n, dt)
+    path_b = grk.grkan_backward_path(x, dy, dx, B, N, d, n_g, m, n, dt)
+
+    def check(st, what):
+        if st != 0:
+            raise grk.GrkanError(st, what)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        check(grk.grkan_forward(x, y, a, b, B, N, d, n_g, m, n, dt, sp), "forward")
+        if ev is not None:
+            ev[1].record(stream)
+        check(grk.grkan_backward_partials(x, dy, a, b, dx, B, N, d, n_g, m, n, dt, ws, wsb, 0, sp),
+              "backward_partials")
+        if ev is not None:
+            ev[2].record(stream)
+        check(grk.grkan_backward_merge(ws, wsb, dA, dB, sums64, B, N, d, n_g, m, n, dt, sp),
+              "backward_merge")
+        if world > 1:
+            dist.all_gather_into_tensor(gathered, sums64)
+            check(grk.grkan_merge_ranks(gathered, world, dA, dB, n_g, m, n, sp), "merge_ranks")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # timed region: exactly K steps between a barrier + synchronize on each side
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid))
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = E * world / (ms_step * 1e-3)
+
+    # end to end through the same ABI calls, host (pinned) buffers in and out
+    y_h = torch.empty_like(x_h, pin_memory=True)
+    dx_h = torch.empty_like(x_h, pin_memory=True)
+    dA_h = torch.empty_like(dA, device="cpu", pin_memory=True)
+    dB_h = torch.empty_like(dB, device="cpu", pin_memory=True)
+
+    def e2e_step():
+        x.copy_(x_h, non_blocking=True)
+        dy.copy_(dy_h, non_blocking=True)
+        step()
+        y_h.copy_(y, non_blocking=True)
+        dx_h.copy_(dx, non_blocking=True)
+        dA_h.copy_(dA, non_blocking=True)
+        dB_h.copy_(dB, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    st, derr = grk.grkan_device_error()
+
+    peak, peak_src = peaks()
+    bwd_bytes = accounting.bytes_per_element("backward", dt) * E
+    fwd_bytes = accounting.bytes_per_element("forward", dt) * E
+    step_bytes = accounting.bytes_per_element("step", dt) * E
+    achieved = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
+        "data": "synthetic (seeded counter-based generator; KAT activation shapes)",
+        "config": dict(w.describe(), global_batch=B * world, seq_len=N,
+                       parallelism="dp%d" % world,
+                       l2="inputs larger than L2 (%.0f MB per tensor), no flush" % (nbytes / 1e6),
+                       kernel_path={"forward": "tma" if path_f == 1 else "generic",
+                                    "backward": "tma" if path_b == 1 else "generic"}),
+        "roofline": {"bound": "hbm", "kernel": "backward stage 1 (dx + dA/dB partials)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                     "bytes_per_launch": bwd_bytes, "launch_ms": bwd_ms},
+        "kernels": {
+            "forward": {"ms": fwd_ms, "GB/s": fwd_bytes / (fwd_ms * 1e-3) / 1e9,
+                        "frac": fwd_bytes / (fwd_ms * 1e-3) / 1e9 / peak},
+            "backward_stage1": {"ms": bwd_ms, "GB/s": achieved, "frac": achieved / peak},
+            "step": {"ms": ms_step, "GB/s": step_bytes / (ms_step * 1e-3) / 1e9,
+                     "frac": step_bytes / (ms_step * 1e-3) / 1e9 / peak,
+                     "frac_of_8TBps": step_bytes / (ms_step * 1e-3) / 8e12},
+        },
+        "e2e": {"value": E * world / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": 2 * nbytes,
+                "d2h_bytes_per_step": 2 * nbytes + (n_g * K) * 4, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * (3 + (1 if world > 1 else 0)),
+        "clocks": clocks,
+        "device_error": derr,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows, el, cores = oracle_rate(w, args.cpu_seconds)
+        s_el = rows * w.d
+        out["cpu_baseline"] = {
+            "value": s_el / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "first %d of %d rows of %s (%d elements), fwd y + bwd dx + dA/dB, %.1f s"
+                      % (rows, w.rows, w.name, s_el, el)}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,45 @@
+"""Algorithmic work of the GR-KAN hot path: bytes that must cross HBM and
+floating-point operations per element.
+
+Bytes (element size es = 4 for float32 I/O, 2 for bf16):
+  forward   read x, write y                   2 es
+  backward  read x and dy, write dx           3 es   (stage 1; the partials,
+            coefficients and the merge add < 1 MB per call and are left out)
+  step      forward + backward                5 es
+Floating point: the forward's extra operations per input are 2m + 2n + 3
+("FlashKAT: Understanding and Addressing Performance Bottlenecks in the
+Kolmogorov-Arnold Transformer", paper notes, section "Insight 2": the GR-KAN
+term (2m+2n+3) d_in next to a linear layer's 2 d_in d_out).
+"""
+
+
+def element_size(dtype):
+    """0 = float32, 1 = bf16."""
+    return 4 if dtype == 0 else 2
+
+
+def bytes_per_element(phase, dtype):
+    es = element_size(dtype)
+    return {"forward": 2 * es, "backward": 3 * es, "step": 5 * es}[phase]
+
+
+def forward_flops_per_element(m, n):
+    return 2 * m + 2 * n + 3
+
+
+def backward_flops_per_element(m, n):
+    """Operations of the backward as this library evaluates it, an FMA counted
+    as two: powers x^2..x^max (max(m, n) - 1 products), P, P', Q, Q' from the
+    powers (2m, 2(m-1), 2n - 1, 2(n-1)), D and the reciprocal (2), y, t,
+    -t y s (3), dx (3), the m+1 + n gradient sums (2(m+1) - 1 + 2n)."""
+    k = max(m, n)
+    powers = max(k - 1, 0)
+    polys = 2 * m + 2 * max(m - 1, 0) + max(2 * n - 1, 0) + 2 * max(n - 1, 0)
+    return powers + polys + 2 + 3 + 3 + (2 * (m + 1) - 1) + 2 * n
+
+
+def flashkat_access_reduction(s_block, d_g):
+    """Factor by which accumulating inside a block before one global update cuts
+    the global accesses for the gradient (section "3. FlashKAT kernel
+    restructuring (Algorithm 2)")."""
+    return s_block * d_g

@@ -1,0 +1,445 @@
+// grkan_api.cu -- the C ABI declared in include/grkan.h: argument checks,
+// work partition, kernel selection and launches. No allocation, no host
+// synchronisation (except grkan_device_error, which says so).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "grkan.h"
+#include "grkan_common.cuh"
+#include "grkan_generic.cuh"
+#include "grkan_merge.cuh"
+#include "grkan_tma.cuh"
+
+namespace {
+
+// Work partition. A "chunk" is SC rows of one group (about 12 KiB of one
+// tensor); a unit (row tile x group) is kChunksPerUnit chunks. The partition
+// depends only on the shape, never on the device, so the float32 partials --
+// and therefore dA and dB -- are the same bits on every run.
+constexpr long long kChunkBytes = 12288;
+constexpr int kChunksPerUnit = 4;
+constexpr int kMaxBoxRows = 256;
+
+struct Plan {
+  long long rows = 0, d = 0, dg = 0;
+  int n_g = 1, m = 0, n = 0, K = 1, es = 4;
+  grkan_dtype_t dtype = GRKAN_F32;
+  int SC = 1;       // rows per chunk
+  int S = 1;        // rows per tile (unit)
+  long long T = 0;  // number of row tiles
+  size_t ws_bytes = 0;
+};
+
+grkan_status_t make_plan(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                         grkan_dtype_t dtype, Plan* p) {
+  if (dtype != GRKAN_F32 && dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
+  if (m < 0 || m > GRKAN_MAX_M || n < 0 || n > GRKAN_MAX_N) return GRKAN_ERR_DEGREE;
+  if (B < 0 || N < 0 || d < 0 || n_g < 1) return GRKAN_ERR_SHAPE;
+  if (d % n_g != 0) return GRKAN_ERR_SHAPE;
+  const long long lim = (1LL << 62);
+  if (B != 0 && N > lim / B) return GRKAN_ERR_SHAPE;
+  const long long rows = (long long)B * N;
+  if (rows != 0 && d > lim / 4 / rows) return GRKAN_ERR_SHAPE;
+  p->rows = rows;
+  p->d = d;
+  p->n_g = n_g;
+  p->dg = d / n_g;
+  p->m = m;
+  p->n = n;
+  p->K = m + 1 + n;
+  p->dtype = dtype;
+  p->es = dtype == GRKAN_F32 ? 4 : 2;
+  const long long row_bytes = p->dg * p->es;
+  long long sc = row_bytes > 0 ? kChunkBytes / row_bytes : kMaxBoxRows;
+  if (sc < 1) sc = 1;
+  if (sc > kMaxBoxRows) sc = kMaxBoxRows;
+  p->SC = (int)sc;
+  p->S = p->SC * kChunksPerUnit;
+  p->T = (rows + p->S - 1) / p->S;
+  if (rows == 0 || d == 0) p->T = 0;
+  p->ws_bytes = (size_t)p->T * (size_t)n_g * (size_t)p->K * sizeof(float);
+  if (p->T > 0 && (long long)n_g * p->T > (1LL << 31) - 1) return GRKAN_ERR_SHAPE;
+  return GRKAN_OK;
+}
+
+bool overlaps(const void* p, size_t pb, const void* q, size_t qb) {
+  if (!p || !q || pb == 0 || qb == 0) return false;
+  const uintptr_t a = (uintptr_t)p, b = (uintptr_t)q;
+  return a < b + qb && b < a + pb;
+}
+
+// Partial overlap is an error; exact aliasing is allowed where documented.
+bool bad_alias(const void* in, const void* out, size_t bytes) {
+  return in != out && overlaps(in, bytes, out, bytes);
+}
+
+bool is_sm100() {
+  static std::once_flag once;
+  static int ok = 0;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaDeviceProp prop;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaGetDeviceProperties(&prop, dev) == cudaSuccess)
+      ok = (prop.major == 10) ? 1 : 0;
+  });
+  return ok != 0;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Dispatch of the generic kernels on the element type.
+template <class IO>
+cudaError_t launch_generic_fwd(const Plan& p, const void* x, void* y, const float* a,
+                               const float* b, cudaStream_t st) {
+  const long long units = p.T * p.n_g;
+  grk::fwd_generic<IO, GRKAN_MAX_M, GRKAN_MAX_N><<<(unsigned)units, grk::kGenericThreads, 0, st>>>(
+      (const typename IO::T*)x, (typename IO::T*)y, a, b, p.rows, p.d, (int)p.dg, p.n_g, p.m, p.n,
+      p.S);
+  return cudaGetLastError();
+}
+
+template <class IO>
+cudaError_t launch_generic_bwd(const Plan& p, const void* x, const void* dy, void* dx,
+                               const float* a, const float* b, float* ws, cudaStream_t st) {
+  const long long units = p.T * p.n_g;
+  grk::bwd_generic<IO, GRKAN_MAX_M, GRKAN_MAX_N><<<(unsigned)units, grk::kGenericThreads, 0, st>>>(
+      (const typename IO::T*)x, (const typename IO::T*)dy, (typename IO::T*)dx, a, b, ws, p.rows,
+      p.d, (int)p.dg, p.n_g, p.m, p.n, p.S, p.T);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const Plan& p, const float* ws, float* dA, float* dB, double* sums64,
+                         cudaStream_t st) {
+  const long long outs = (long long)p.n_g * p.K;
+  const unsigned blocks = (unsigned)((outs + grk::kMergeWarps - 1) / grk::kMergeWarps);
+  grk::merge_partials<<<blocks, grk::kMergeWarps * 32, 0, st>>>(ws, dA, dB, sums64, p.T, p.n_g,
+                                                                 p.m, p.n);
+  return cudaGetLastError();
+}
+
+// --- path selection ----------------------------------------------------------
+
+bool tma_degree_supported(int m, int n) { return grk::tma_has_degree(m, n); }
+
+// Box width for the TMA tensor maps: the largest divisor of d_g that is at most
+// 256 elements with a whole number of 16-byte units. 0 if none.
+int tma_box_width(const Plan& p) {
+  if (p.dg <= 0) return 0;
+  for (long long w = p.dg < 256 ? p.dg : 256; w >= 1; --w) {
+    if (p.dg % w == 0 && (w * p.es) % 16 == 0) return (int)w;
+  }
+  return 0;
+}
+
+bool tma_shape_ok(const Plan& p) {
+  if (p.rows <= 0 || p.d <= 0) return false;
+  if ((p.d * p.es) % 16 != 0 || (p.dg * p.es) % 16 != 0) return false;
+  if (p.rows > 0x7fffffffLL || p.d > 0x7fffffffLL) return false;
+  const int bw = tma_box_width(p);
+  if (bw == 0) return false;
+  // a chunk (SC rows x d_g) fits one stage, and every TMA box inside it starts
+  // on a 128-byte boundary of shared memory
+  if ((long long)p.SC * p.dg * p.es > (long long)grk::kMaxChunkBytes) return false;
+  return ((long long)p.SC * bw * p.es) % 128 == 0;
+}
+
+int choose_fwd_path(const Plan& p, const void* x, const void* y, uint32_t flags) {
+  if (flags & GRKAN_FLAG_GENERIC) return 0;
+  if (!tma_degree_supported(p.m, p.n) || !tma_shape_ok(p)) return 0;
+  if (!aligned16(x) || !aligned16(y)) return 0;
+  return 1;
+}
+
+int choose_bwd_path(const Plan& p, const void* x, const void* dy, const void* dx,
+                    uint32_t flags) {
+  if (flags & GRKAN_FLAG_GENERIC) return 0;
+  if (!tma_degree_supported(p.m, p.n) || !tma_shape_ok(p)) return 0;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return 0;
+  return 1;
+}
+
+// --- TMA tensor maps -----------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// 2-D map over the (rows, d) tensor, box = (bw columns, SC rows).
+bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)p.d, (cuuint64_t)p.rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(p.d * p.es)};
+  const cuuint32_t box[2] = {(cuuint32_t)bw, (cuuint32_t)p.SC};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      p.dtype == GRKAN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+grk::TmaGeom make_geom(const Plan& p, int bw) {
+  grk::TmaGeom g;
+  g.rows = p.rows;
+  g.dg = (int)p.dg;
+  g.n_g = p.n_g;
+  g.SC = p.SC;
+  g.chunks_per_unit = kChunksPerUnit;
+  g.T = p.T;
+  g.bw = bw;
+  g.nbox = (int)(p.dg / bw);
+  g.chunk_bytes = (unsigned)(p.SC * p.dg * p.es);
+  g.m = p.m;
+  g.n = p.n;
+  return g;
+}
+
+int sm_count() {
+  static std::once_flag once;
+  static int sms = 148;
+  std::call_once(once, [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      sms = v;
+  });
+  return sms;
+}
+
+grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float* a,
+                              const float* b, cudaStream_t st) {
+  const int bw = tma_box_width(p);
+  CUtensorMap mx, my;
+  if (!make_map(&mx, x, p, bw) || !make_map(&my, y, p, bw)) return GRKAN_ERR_CUDA;
+  const grk::TmaGeom geom = make_geom(p, bw);
+  cudaError_t e = grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, my, a, b, sm_count(), st);
+  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx,
+                              const float* a, const float* b, float* ws, cudaStream_t st) {
+  const int bw = tma_box_width(p);
+  CUtensorMap mx, mdy, mdx;
+  if (!make_map(&mx, x, p, bw) || !make_map(&mdy, dy, p, bw) || !make_map(&mdx, dx, p, bw))
+    return GRKAN_ERR_CUDA;
+  const grk::TmaGeom geom = make_geom(p, bw);
+  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, mdx, a, b, ws,
+                                      sm_count(), st);
+  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+grkan_status_t check_coef_ptrs(const Plan& p, const float* a, const float* b) {
+  if (!a) return GRKAN_ERR_NULL;
+  if (p.n > 0 && !b) return GRKAN_ERR_NULL;
+  return GRKAN_OK;
+}
+
+grkan_status_t do_forward(const void* x, void* y, const float* a, const float* b, int64_t B,
+                          int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                          grkan_dtype_t dtype, uint32_t flags, void* stream) {
+  if (flags & ~GRKAN_FLAG_GENERIC) return GRKAN_ERR_FLAGS;
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (p.rows == 0 || p.d == 0) return GRKAN_OK;
+  if (!x || !y) return GRKAN_ERR_NULL;
+  if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+  const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
+  if (bad_alias(x, y, bytes)) return GRKAN_ERR_ALIAS;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (choose_fwd_path(p, x, y, flags) == 1) return launch_tma_fwd(p, x, y, a, b, st);
+  cudaError_t e = (dtype == GRKAN_F32) ? launch_generic_fwd<grk::IoF32>(p, x, y, a, b, st)
+                                       : launch_generic_fwd<grk::IoBF16>(p, x, y, a, b, st);
+  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const float* a,
+                           const float* b, void* dx, void* ws, size_t ws_bytes, uint32_t flags,
+                           cudaStream_t st) {
+  if (!x || !dy || !dx) return GRKAN_ERR_NULL;
+  grkan_status_t s = check_coef_ptrs(p, a, b);
+  if (s != GRKAN_OK) return s;
+  if (!ws || ws_bytes < p.ws_bytes || !aligned16(ws)) return GRKAN_ERR_WORKSPACE;
+  const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
+  if (bad_alias(x, dx, bytes) || bad_alias(dy, dx, bytes)) return GRKAN_ERR_ALIAS;
+  if (overlaps(ws, p.ws_bytes, x, bytes) || overlaps(ws, p.ws_bytes, dy, bytes) ||
+      overlaps(ws, p.ws_bytes, dx, bytes))
+    return GRKAN_ERR_ALIAS;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  if (choose_bwd_path(p, x, dy, dx, flags) == 1)
+    return launch_tma_bwd(p, x, dy, dx, a, b, (float*)ws, st);
+  cudaError_t e =
+      (p.dtype == GRKAN_F32)
+          ? launch_generic_bwd<grk::IoF32>(p, x, dy, dx, a, b, (float*)ws, st)
+          : launch_generic_bwd<grk::IoBF16>(p, x, dy, dx, a, b, (float*)ws, st);
+  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+grkan_status_t do_merge(const Plan& p, const void* ws, size_t ws_bytes, float* dA, float* dB,
+                        double* sums64, cudaStream_t st) {
+  if (!dA || (p.n > 0 && !dB)) return GRKAN_ERR_NULL;
+  if (p.T > 0 && (!ws || ws_bytes < p.ws_bytes)) return GRKAN_ERR_WORKSPACE;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  cudaError_t e = launch_merge(p, (const float*)ws, dA, dB, sums64, st);
+  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+grkan_status_t grkan_forward(const void* x, void* y, const float* a, const float* b, int64_t B,
+                             int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                             grkan_dtype_t dtype, void* stream) {
+  return do_forward(x, y, a, b, B, N, d, n_g, m, n, dtype, 0u, stream);
+}
+
+grkan_status_t grkan_forward_ex(const void* x, void* y, const float* a, const float* b, int64_t B,
+                                int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                                grkan_dtype_t dtype, uint32_t flags, void* stream) {
+  return do_forward(x, y, a, b, B, N, d, n_g, m, n, dtype, flags, stream);
+}
+
+size_t grkan_backward_workspace_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
+                                      int32_t n, grkan_dtype_t dtype) {
+  Plan p;
+  if (make_plan(B, N, d, n_g, m, n, dtype, &p) != GRKAN_OK) return 0;
+  return p.ws_bytes;
+}
+
+grkan_status_t grkan_backward_partials(const void* x, const void* dy, const float* a,
+                                       const float* b, void* dx, int64_t B, int64_t N, int64_t d,
+                                       int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                                       void* workspace, size_t workspace_bytes, uint32_t flags,
+                                       void* stream) {
+  if (flags & ~GRKAN_FLAG_GENERIC) return GRKAN_ERR_FLAGS;
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (p.T == 0) return GRKAN_OK;
+  return do_partials(p, x, dy, a, b, dx, workspace, workspace_bytes, flags,
+                     (cudaStream_t)stream);
+}
+
+grkan_status_t grkan_backward_merge(const void* workspace, size_t workspace_bytes, float* dA,
+                                    float* dB, double* sums64, int64_t B, int64_t N, int64_t d,
+                                    int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                                    void* stream) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  return do_merge(p, workspace, workspace_bytes, dA, dB, sums64, (cudaStream_t)stream);
+}
+
+grkan_status_t grkan_backward_ex(const void* x, const void* dy, const float* a, const float* b,
+                                 void* dx, float* dA, float* dB, int64_t B, int64_t N, int64_t d,
+                                 int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                                 void* workspace, size_t workspace_bytes, uint32_t flags,
+                                 void* stream) {
+  if (flags & ~GRKAN_FLAG_GENERIC) return GRKAN_ERR_FLAGS;
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (!dA || (p.n > 0 && !dB)) return GRKAN_ERR_NULL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.T > 0) {
+    s = do_partials(p, x, dy, a, b, dx, workspace, workspace_bytes, flags, st);
+    if (s != GRKAN_OK) return s;
+  }
+  return do_merge(p, workspace, workspace_bytes, dA, dB, nullptr, st);
+}
+
+grkan_status_t grkan_backward(const void* x, const void* dy, const float* a, const float* b,
+                              void* dx, float* dA, float* dB, int64_t B, int64_t N, int64_t d,
+                              int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  return grkan_backward_ex(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, workspace,
+                           workspace_bytes, 0u, stream);
+}
+
+grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* dA, float* dB,
+                                 int32_t n_g, int32_t m, int32_t n, void* stream) {
+  if (m < 0 || m > GRKAN_MAX_M || n < 0 || n > GRKAN_MAX_N) return GRKAN_ERR_DEGREE;
+  if (n_g < 1 || world < 1) return GRKAN_ERR_SHAPE;
+  if (!gathered || !dA || (n > 0 && !dB)) return GRKAN_ERR_NULL;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  const long long per = (long long)n_g * (m + 1 + n);
+  const unsigned threads = 128;
+  grk::merge_ranks<<<(unsigned)((per + threads - 1) / threads), threads, 0,
+                     (cudaStream_t)stream>>>(gathered, world, dA, dB, n_g, m, n);
+  return cudaGetLastError() == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+int32_t grkan_forward_path(const void* x, const void* y, int64_t B, int64_t N, int64_t d,
+                           int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                           uint32_t flags) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return -(int32_t)s;
+  if (flags & ~GRKAN_FLAG_GENERIC) return -(int32_t)GRKAN_ERR_FLAGS;
+  return choose_fwd_path(p, x, y, flags);
+}
+
+int32_t grkan_backward_path(const void* x, const void* dy, const void* dx, int64_t B, int64_t N,
+                            int64_t d, int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                            uint32_t flags) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return -(int32_t)s;
+  if (flags & ~GRKAN_FLAG_GENERIC) return -(int32_t)GRKAN_ERR_FLAGS;
+  return choose_bwd_path(p, x, dy, dx, flags);
+}
+
+grkan_status_t grkan_device_error(uint32_t* code, void* stream) {
+  if (!code) return GRKAN_ERR_NULL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (grk::read_device_error(code, st) != cudaSuccess) return GRKAN_ERR_CUDA;
+  return GRKAN_OK;
+}
+
+grkan_status_t grkan_clear_device_error(void* stream) {
+  return grk::clear_device_error((cudaStream_t)stream) == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+}
+
+const char* grkan_status_string(grkan_status_t s) {
+  switch (s) {
+    case GRKAN_OK: return "GRKAN_OK";
+    case GRKAN_ERR_NULL: return "GRKAN_ERR_NULL: a required pointer is NULL";
+    case GRKAN_ERR_SHAPE: return "GRKAN_ERR_SHAPE: invalid sizes or d % n_g != 0";
+    case GRKAN_ERR_DEGREE: return "GRKAN_ERR_DEGREE: m or n out of range";
+    case GRKAN_ERR_DTYPE: return "GRKAN_ERR_DTYPE: unknown dtype";
+    case GRKAN_ERR_WORKSPACE: return "GRKAN_ERR_WORKSPACE: workspace missing, small or unaligned";
+    case GRKAN_ERR_CUDA: return "GRKAN_ERR_CUDA: CUDA error while enqueueing";
+    case GRKAN_ERR_ALIAS: return "GRKAN_ERR_ALIAS: partially overlapping input and output";
+    case GRKAN_ERR_FLAGS: return "GRKAN_ERR_FLAGS: unknown flag bits";
+    case GRKAN_ERR_DEVICE: return "GRKAN_ERR_DEVICE: current device is not sm_100";
+  }
+  return "GRKAN_ERR_UNKNOWN";
+}
+
+int32_t grkan_abi_version(void) { return GRKAN_ABI_VERSION; }
+
+}  // extern "C"

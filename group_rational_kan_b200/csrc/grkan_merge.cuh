@@ -1,0 +1,62 @@
+// grkan_merge.cuh -- second stage of the coefficient-gradient reduction.
+//
+// The first stage leaves one float32 partial per (row tile, group,
+// coefficient). This kernel adds the T partials of each (group, coefficient)
+// in double precision in a fixed order -- lane l takes tiles l, l+32, ...,
+// then a fixed xor butterfly -- and writes dA / dB. This is the "single
+// controllable merge step" that replaces scattered atomic updates ("PolyKAN:
+// Efficient Fused GPU Operators for Polynomial Kolmogorov-Arnold Network
+// Variants", abstract, technique (iii)); the order never depends on timing,
+// so the result is identical from run to run.
+#pragma once
+
+#include "grkan_common.cuh"
+
+namespace grk {
+
+constexpr int kMergeWarps = 4;
+
+__global__ void __launch_bounds__(kMergeWarps * 32)
+merge_partials(const float* __restrict__ ws, float* __restrict__ dA, float* __restrict__ dB,
+               double* __restrict__ sums64, long long T, int n_g, int m, int n) {
+  const int K = m + 1 + n;
+  const int lane = threadIdx.x & 31;
+  const long long o = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+  if (o >= (long long)n_g * K) return;
+  const float* p = ws + o * T;
+  double s = 0.0;
+  for (long long t = lane; t < T; t += 32) s += (double)p[t];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) {
+    const int g = (int)(o / K);
+    const int k = (int)(o - (long long)g * K);
+    if (k <= m)
+      dA[(long long)g * (m + 1) + k] = (float)s;
+    else
+      dB[(long long)g * n + (k - m - 1)] = (float)s;
+    if (sums64) sums64[o] = s;
+  }
+}
+
+// Data-parallel merge across devices: gathered holds `world` blocks of
+// n_g * K float64 sums in rank order (one block per device, e.g. after an
+// all-gather). Adds them in rank order and writes dA / dB.
+__global__ void merge_ranks(const double* __restrict__ gathered, int world,
+                            float* __restrict__ dA, float* __restrict__ dB, int n_g, int m,
+                            int n) {
+  const int K = m + 1 + n;
+  const long long per = (long long)n_g * K;
+  const long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= per) return;
+  double s = 0.0;
+  for (int r = 0; r < world; ++r) s += gathered[(long long)r * per + o];
+  const int g = (int)(o / K);
+  const int k = (int)(o - (long long)g * K);
+  if (k <= m)
+    dA[(long long)g * (m + 1) + k] = (float)s;
+  else
+    dB[(long long)g * n + (k - m - 1)] = (float)s;
+}
+
+}  // namespace grk

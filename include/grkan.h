@@ -1,0 +1,174 @@
+/*
+ * grkan.h -- C ABI of the B200 (sm_100a) GR-KAN group-rational activation.
+ *
+ * The operation. The Kolmogorov-Arnold Transformer replaces the MLP's fixed
+ * activation by a Group-Rational KAN: channels are split into n_g groups and
+ * every group shares the coefficients of one "safe" Pade activation unit
+ * ("FlashKAT: Understanding and Addressing Performance Bottlenecks in the
+ * Kolmogorov-Arnold Transformer", paper notes, section "KAT's breakthrough and
+ * remaining problem"; 8 groups, 6 numerator and 4 denominator coefficients in
+ * section "Loss / training strategy"):
+ *
+ *   x : row-major (B, N, d) tensor, rows = B*N; channel c is in group
+ *       g = c / d_g with d_g = d / n_g (contiguous channel blocks)
+ *   P(x) = a[g][0] + a[g][1] x + ... + a[g][m] x^m
+ *   Q(x) = b[g][0] x + b[g][1] x^2 + ... + b[g][n-1] x^n   (b_1..b_n, no b_0)
+ *   y    = P(x) / (1 + |Q(x)|)
+ *
+ * The backward pass (gradient equations cited, not printed, in section
+ * "2. The atomic-add problem of the original KAT"; derived here by calculus,
+ * with D = 1 + |Q|, s = sign(Q), sign(0) = 0, g = dL/dy):
+ *   dx        = g (P'(x) - y s Q'(x)) / D
+ *   dA[g][i]  = sum over every row and every channel of group g of  g x^i / D
+ *   dB[g][j]  = sum over the same elements of  -g y s x^(j+1) / D
+ * The sums run over all batch x sequence x in-group elements (same section).
+ * They are computed without atomics, in two stages (cf. the two-stage reduction
+ * of "PolyKAN: Efficient Fused GPU Operators for Polynomial Kolmogorov-Arnold
+ * Network Variants", abstract, technique (iii)): per (row tile, group) partial
+ * sums into a caller-owned workspace, then a fixed-order merge in double
+ * precision. dA and dB are therefore bit-identical from run to run for a given
+ * shape and a given pointer alignment class (16-byte aligned or not).
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named x, y, dy, dx, a, b, dA, dB, workspace are DEVICE pointers
+ *    (or managed memory) of the current CUDA device; the caller owns them.
+ *    The library allocates no memory and keeps no per-call state.
+ *  - dtype selects the element type of x, y, dy, dx: float32 or bfloat16.
+ *    Coefficients a (n_g x (m+1)), b (n_g x n) and gradients dA, dB are always
+ *    float32, row-major. Arithmetic is float32; the merge is float64.
+ *  - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous: it validates, enqueues kernels and returns.
+ *  - 0 <= m <= GRKAN_MAX_M, 0 <= n <= GRKAN_MAX_N, n_g >= 1, d % n_g == 0.
+ *    With n = 0, b may be NULL and Q = 0. B*N*d == 0 is a valid no-op
+ *    (the backward then writes zeros to dA and dB).
+ *  - Aliasing: y may equal x (in place) and dx may equal dy or x; any other
+ *    overlap between an input and an output returns GRKAN_ERR_ALIAS.
+ *  - Errors are returned, never thrown; on error nothing is enqueued.
+ *    GRKAN_ERR_CUDA reports a launch failure (cudaGetLastError); a fault that
+ *    happens later on the GPU surfaces at the caller's next synchronisation.
+ */
+#ifndef GRKAN_H
+#define GRKAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GRKAN_API __attribute__((visibility("default")))
+#else
+#define GRKAN_API
+#endif
+
+#define GRKAN_ABI_VERSION 1
+#define GRKAN_MAX_M 8
+#define GRKAN_MAX_N 8
+
+typedef enum grkan_dtype { GRKAN_F32 = 0, GRKAN_BF16 = 1 } grkan_dtype_t;
+
+typedef enum grkan_status {
+  GRKAN_OK = 0,
+  GRKAN_ERR_NULL = 1,      /* a required pointer is NULL */
+  GRKAN_ERR_SHAPE = 2,     /* negative size, n_g < 1, d % n_g != 0, or size overflow */
+  GRKAN_ERR_DEGREE = 3,    /* m or n outside [0, GRKAN_MAX_M] / [0, GRKAN_MAX_N] */
+  GRKAN_ERR_DTYPE = 4,     /* unknown dtype */
+  GRKAN_ERR_WORKSPACE = 5, /* workspace NULL or smaller than the query says */
+  GRKAN_ERR_CUDA = 6,      /* CUDA reported an error while enqueueing */
+  GRKAN_ERR_ALIAS = 7,     /* partially overlapping input and output */
+  GRKAN_ERR_FLAGS = 8,     /* unknown flag bits */
+  GRKAN_ERR_DEVICE = 9     /* the current device is not sm_100 (B200 class) */
+} grkan_status_t;
+
+/* Flag bits for the *_ex entry points. */
+#define GRKAN_FLAG_GENERIC 1u /* use the plain grid-stride kernels even where the
+                                 TMA-pipelined kernels apply (for testing) */
+
+/* Forward: y = P(x) / (1 + |Q(x)|) elementwise, group coefficients a, b. */
+GRKAN_API grkan_status_t grkan_forward(const void* x, void* y, const float* a, const float* b, int64_t B,
+                             int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                             grkan_dtype_t dtype, void* stream);
+
+GRKAN_API grkan_status_t grkan_forward_ex(const void* x, void* y, const float* a, const float* b, int64_t B,
+                                int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                                grkan_dtype_t dtype, uint32_t flags, void* stream);
+
+/* Bytes of device workspace grkan_backward needs for this shape (0 when the
+ * input is empty). The layout is private; its size depends only on the shape. */
+GRKAN_API size_t grkan_backward_workspace_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
+                                      int32_t n, grkan_dtype_t dtype);
+
+/* Backward: dx (same shape and dtype as x), dA (n_g x (m+1)) and dB (n_g x n),
+ * both overwritten (not accumulated). workspace must hold at least
+ * grkan_backward_workspace_bytes(...) bytes, 16-byte aligned; its previous
+ * contents do not matter. Equivalent to grkan_backward_partials followed by
+ * grkan_backward_merge on the same stream. */
+GRKAN_API grkan_status_t grkan_backward(const void* x, const void* dy, const float* a, const float* b,
+                              void* dx, float* dA, float* dB, int64_t B, int64_t N, int64_t d,
+                              int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+GRKAN_API grkan_status_t grkan_backward_ex(const void* x, const void* dy, const float* a, const float* b,
+                                 void* dx, float* dA, float* dB, int64_t B, int64_t N, int64_t d,
+                                 int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                                 void* workspace, size_t workspace_bytes, uint32_t flags,
+                                 void* stream);
+
+/* Stage 1 alone: dx, plus one float32 partial sum per (row tile, group,
+ * coefficient) into the workspace. */
+GRKAN_API grkan_status_t grkan_backward_partials(const void* x, const void* dy, const float* a,
+                                       const float* b, void* dx, int64_t B, int64_t N, int64_t d,
+                                       int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                                       void* workspace, size_t workspace_bytes, uint32_t flags,
+                                       void* stream);
+
+/* Stage 2 alone: fixed-order float64 sum of the workspace partials written by
+ * grkan_backward_partials for the same shape; writes dA and dB (float32).
+ * If sums64 is not NULL it also receives the float64 sums, laid out
+ * [n_g][m+1+n] (a_0..a_m then b_1..b_n), for a later cross-device merge. */
+GRKAN_API grkan_status_t grkan_backward_merge(const void* workspace, size_t workspace_bytes, float* dA,
+                                    float* dB, double* sums64, int64_t B, int64_t N, int64_t d,
+                                    int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                                    void* stream);
+
+/* Data-parallel merge across devices. Each device runs the backward on its
+ * own rows and grkan_backward_merge with sums64; the caller gathers the
+ * world blocks of n_g*(m+1+n) float64 sums into `gathered` in rank order (for
+ * example with an all-gather). This adds them in rank order -- the same order
+ * on every device, independent of the transport -- and writes dA and dB
+ * (float32), so all devices hold bit-identical gradients. gathered, dA and dB
+ * are device pointers; world >= 1. */
+GRKAN_API grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* dA,
+                                           float* dB, int32_t n_g, int32_t m, int32_t n,
+                                           void* stream);
+
+/* Which kernels a call with these arguments would run: 1 = TMA-pipelined
+ * persistent kernels, 0 = generic grid-stride kernels, < 0 = invalid arguments
+ * (the negated status). x, y are only inspected for alignment. */
+GRKAN_API int32_t grkan_forward_path(const void* x, const void* y, int64_t B, int64_t N, int64_t d,
+                           int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype, uint32_t flags);
+GRKAN_API int32_t grkan_backward_path(const void* x, const void* dy, const void* dx, int64_t B, int64_t N,
+                            int64_t d, int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype,
+                            uint32_t flags);
+
+/* Device-side error word. The pipelined kernels bound every wait; a wait that
+ * runs out (which correct inputs never cause) sets a nonzero code here and the
+ * kernel returns early instead of hanging. grkan_device_error copies the word
+ * to *code (host pointer) and synchronises the stream; grkan_clear_device_error
+ * resets it (stream-ordered). */
+GRKAN_API grkan_status_t grkan_device_error(uint32_t* code, void* stream);
+GRKAN_API grkan_status_t grkan_clear_device_error(void* stream);
+
+/* Human-readable name of a status code (static string). */
+GRKAN_API const char* grkan_status_string(grkan_status_t status);
+
+/* GRKAN_ABI_VERSION of the built library. */
+GRKAN_API int32_t grkan_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRKAN_H */

@@ -1,0 +1,131 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/grkan.h declares, and rejects bad arguments with the documented codes
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import group_rational_kan_b200 as grk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "grkan.h")
+
+OK, NULL, SHAPE, DEGREE, DTYPE, WORKSPACE, CUDA, ALIAS, FLAGS, DEVICE = range(10)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GRKAN_API\s+[\w\s\*]+?\b(grkan_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for need in ("grkan_forward", "grkan_backward", "grkan_backward_workspace_bytes",
+                 "grkan_status_string"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(grk.library_path if os.path.exists(grk.library_path) else grk.lib()._name)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert grk.grkan_abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(10):
+        s = grk.grkan_status_string(code)
+        assert s.startswith("GRKAN_")
+    assert "UNKNOWN" in grk.grkan_status_string(99)
+
+
+def test_workspace_bytes():
+    # KAT-B: d_g = 384 bf16 -> 16 rows per chunk, 64 rows per tile, 1576 tiles
+    assert grk.grkan_backward_workspace_bytes(512, 197, 3072, 8, 5, 4, grk.BF16) == 1576 * 8 * 10 * 4
+    # KAT-T: d_g = 96 f32 -> 32 rows per chunk, 128 per tile, 1576 tiles
+    assert grk.grkan_backward_workspace_bytes(1024, 197, 768, 8, 5, 4, grk.F32) == 1576 * 8 * 10 * 4
+    assert grk.grkan_backward_workspace_bytes(0, 197, 768, 8, 5, 4, grk.F32) == 0
+    assert grk.grkan_backward_workspace_bytes(2, 3, 10, 3, 5, 4, grk.F32) == 0  # d % n_g != 0
+    assert grk.grkan_backward_workspace_bytes(2, 3, 12, 3, 9, 4, grk.F32) == 0  # degree
+
+
+def test_path_selection():
+    A = 1 << 20  # an aligned fake address, never dereferenced
+    kat_b = (512, 197, 3072, 8, 5, 4, grk.BF16)
+    assert grk.grkan_forward_path(A, A, *kat_b) == 1
+    assert grk.grkan_backward_path(A, A, A, *kat_b) == 1
+    assert grk.grkan_backward_path(A, A, A, *kat_b, flags=grk.FLAG_GENERIC) == 0
+    assert grk.grkan_backward_path(A + 4, A, A, *kat_b) == 0  # unaligned -> generic
+    assert grk.grkan_forward_path(A, A, 2, 3, 30, 3, 5, 4, grk.F32) == 0  # 40-byte groups
+    assert grk.grkan_forward_path(A, A, 2, 3, 48, 4, 3, 2, grk.F32) == 0  # other degree
+    assert grk.grkan_forward_path(A, A, 2, 16, 64, 8, 5, 4, grk.F32) == 1  # tiny
+    assert grk.grkan_forward_path(A, A, 256, 197, 3072, 1, 5, 4, grk.F32) == 1  # n_g = 1
+    assert grk.grkan_forward_path(A, A, 256, 197, 3072, 64, 5, 4, grk.F32) == 1  # n_g = 64
+    assert grk.grkan_forward_path(A, A, 2, 3, 12, 5, 5, 4, grk.F32) == -SHAPE
+    assert grk.grkan_forward_path(A, A, 2, 3, 12, 3, 5, 4, 7) == -DTYPE
+    assert grk.grkan_forward_path(A, A, 2, 3, 12, 3, 5, 4, grk.F32, flags=8) == -FLAGS
+
+
+def test_argument_errors_need_no_gpu():
+    A = 1 << 20
+    f = grk.grkan_forward_ex
+    shape = (2, 3, 12, 3, 5, 4, grk.F32)
+    assert f(None, A, A, A, *shape, 0, 0) == NULL
+    assert f(A, None, A, A, *shape, 0, 0) == NULL
+    assert f(A, A, None, A, *shape, 0, 0) == NULL
+    assert f(A, A, A, None, *shape, 0, 0) == NULL
+    assert f(A, A, A, None, 2, 3, 12, 3, 5, 0, grk.F32, 0, 0) != NULL  # n = 0: b may be NULL
+    assert f(A, A, A, A, 2, 3, 12, 5, 5, 4, grk.F32, 0, 0) == SHAPE
+    assert f(A, A, A, A, -1, 3, 12, 3, 5, 4, grk.F32, 0, 0) == SHAPE
+    assert f(A, A, A, A, 2, 3, 12, 0, 5, 4, grk.F32, 0, 0) == SHAPE
+    assert f(A, A, A, A, 2, 3, 12, 3, 9, 4, grk.F32, 0, 0) == DEGREE
+    assert f(A, A, A, A, 2, 3, 12, 3, 5, -1, grk.F32, 0, 0) == DEGREE
+    assert f(A, A, A, A, 2, 3, 12, 3, 5, 4, 3, 0, 0) == DTYPE
+    assert f(A, A, A, A, *shape, 2, 0) == FLAGS
+    assert f(A, A + 4, A, A, *shape, 0, 0) == ALIAS  # partial overlap
+    assert f(A, A, A, A, 1 << 40, 1 << 40, 12, 3, 5, 4, grk.F32, 0, 0) == SHAPE  # overflow
+    assert f(None, None, None, None, 0, 3, 12, 3, 5, 4, grk.F32, 0, 0) == OK  # empty: no-op
+    # everything valid but no sm_100 device here
+    if not _has_gpu():
+        assert f(A, A, A, A, *shape, 0, 0) == DEVICE
+
+
+def test_backward_argument_errors_need_no_gpu():
+    A = 1 << 20
+    W = 1 << 30
+    shape = (2, 3, 12, 3, 5, 4, grk.F32)
+    need = grk.grkan_backward_workspace_bytes(*shape)
+    assert need > 0
+    b = grk.grkan_backward_ex
+    assert b(A, A, A, A, A, None, A, *shape, W, need, 0, 0) == NULL
+    assert b(A, A, A, A, A, A, None, *shape, W, need, 0, 0) == NULL
+    assert b(A, A, A, A, A, A, A, *shape, None, need, 0, 0) == WORKSPACE
+    assert b(A, A, A, A, A, A, A, *shape, W, need - 4, 0, 0) == WORKSPACE
+    assert b(A, A, A, A, A, A, A, *shape, W + 4, need, 0, 0) == WORKSPACE  # unaligned
+    assert b(A, A, A, A, A + 8, A, A, *shape, W, need, 0, 0) == ALIAS
+    assert b(A, A, A, A, A, A, A, *shape, A + 16, need, 0, 0) == ALIAS  # workspace inside x
+    assert b(A, A, A, A, A, A, A, *shape, W, need, 4, 0) == FLAGS
+    if not _has_gpu():
+        assert b(A, A, A, A, A, A, A, *shape, W, need, 0, 0) == DEVICE
+
+
+def _has_gpu():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The binding has no CPU fallback: a missing library is an ImportError."""
+    import importlib
+    import group_rational_kan_b200.build as b
+    monkeypatch.setattr(grk, "_lib", None)
+    monkeypatch.setattr(grk, "library_path", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(b, "needs_build", lambda: False)
+    with pytest.raises(ImportError):
+        grk.lib()
+    importlib.reload(grk)
