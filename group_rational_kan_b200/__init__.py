@@ -18,7 +18,7 @@ __all__ = [
     "grkan_backward_partials", "grkan_backward_merge", "grkan_backward_workspace_bytes",
     "grkan_merge_ranks",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
-    "grkan_status_string", "grkan_abi_version", "forward", "backward", "workspace_bytes",
+    "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
 ]
 
 F32, BF16 = 0, 1
@@ -34,7 +34,10 @@ _lock = threading.Lock()
 class GrkanError(RuntimeError):
     def __init__(self, status, what=""):
         self.status = status
-        super().__init__("%s%s" % (what + ": " if what else "", grkan_status_string(status)))
+        msg = grkan_status_string(status)
+        if status == 6:  # GRKAN_ERR_CUDA: add the failing CUDA call
+            msg += " [%s]" % grkan_last_error()
+        super().__init__("%s%s" % (what + ": " if what else "", msg))
 
 
 def _load():
@@ -66,6 +69,7 @@ def _load():
         "grkan_clear_device_error": (S, [P]),
         "grkan_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "grkan_abi_version": (I32, []),
+        "grkan_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -180,6 +184,10 @@ def grkan_status_string(status):
 
 def grkan_abi_version():
     return lib().grkan_abi_version()
+
+
+def grkan_last_error():
+    return lib().grkan_last_error().decode()
 
 
 # --- conveniences (torch tensors in, torch tensors out) ------------------------

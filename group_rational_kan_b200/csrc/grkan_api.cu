@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <atomic>
@@ -16,6 +17,20 @@
 #include "grkan_tma.cuh"
 
 namespace {
+
+thread_local char g_last_error[256] = "no error";
+
+void set_last_error(const char* where, const char* what, int code) {
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s (%d)", where, what, code);
+}
+
+// GRKAN_OK, or GRKAN_ERR_CUDA with the failing call recorded for
+// grkan_last_error().
+grkan_status_t cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return GRKAN_OK;
+  set_last_error(where, cudaGetErrorString(e), (int)e);
+  return GRKAN_ERR_CUDA;
+}
 
 // Work partition. A "chunk" is SC rows of one group (about 12 KiB of one
 // tensor); a unit (row tile x group) is kChunksPerUnit chunks. The partition
@@ -187,7 +202,10 @@ EncodeTiledFn encode_fn() {
 // 2-D map over the (rows, d) tensor, box = (bw columns, SC rows).
 bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
+  if (!fn) {
+    set_last_error("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled not found", 0);
+    return false;
+  }
   const cuuint64_t dims[2] = {(cuuint64_t)p.d, (cuuint64_t)p.rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(p.d * p.es)};
   const cuuint32_t box[2] = {(cuuint32_t)bw, (cuuint32_t)p.SC};
@@ -197,6 +215,7 @@ bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
   CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) set_last_error("cuTensorMapEncodeTiled", "failed", (int)r);
   return r == CUDA_SUCCESS;
 }
 
@@ -235,7 +254,7 @@ grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float
   if (!make_map(&mx, x, p, bw) || !make_map(&my, y, p, bw)) return GRKAN_ERR_CUDA;
   const grk::TmaGeom geom = make_geom(p, bw);
   cudaError_t e = grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, my, a, b, sm_count(), st);
-  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(e, "forward (TMA) launch");
 }
 
 grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx,
@@ -247,7 +266,7 @@ grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void
   const grk::TmaGeom geom = make_geom(p, bw);
   cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, mdx, a, b, ws,
                                       sm_count(), st);
-  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(e, "backward (TMA) launch");
 }
 
 grkan_status_t check_coef_ptrs(const Plan& p, const float* a, const float* b) {
@@ -273,7 +292,7 @@ grkan_status_t do_forward(const void* x, void* y, const float* a, const float* b
   if (choose_fwd_path(p, x, y, flags) == 1) return launch_tma_fwd(p, x, y, a, b, st);
   cudaError_t e = (dtype == GRKAN_F32) ? launch_generic_fwd<grk::IoF32>(p, x, y, a, b, st)
                                        : launch_generic_fwd<grk::IoBF16>(p, x, y, a, b, st);
-  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(e, "forward (generic) launch");
 }
 
 grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const float* a,
@@ -295,7 +314,7 @@ grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const f
       (p.dtype == GRKAN_F32)
           ? launch_generic_bwd<grk::IoF32>(p, x, dy, dx, a, b, (float*)ws, st)
           : launch_generic_bwd<grk::IoBF16>(p, x, dy, dx, a, b, (float*)ws, st);
-  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(e, "backward (generic) launch");
 }
 
 grkan_status_t do_merge(const Plan& p, const void* ws, size_t ws_bytes, float* dA, float* dB,
@@ -304,7 +323,7 @@ grkan_status_t do_merge(const Plan& p, const void* ws, size_t ws_bytes, float* d
   if (p.T > 0 && (!ws || ws_bytes < p.ws_bytes)) return GRKAN_ERR_WORKSPACE;
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
   cudaError_t e = launch_merge(p, (const float*)ws, dA, dB, sums64, st);
-  return e == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(e, "merge launch");
 }
 
 }  // namespace
@@ -390,7 +409,7 @@ grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* d
   const unsigned threads = 128;
   grk::merge_ranks<<<(unsigned)((per + threads - 1) / threads), threads, 0,
                      (cudaStream_t)stream>>>(gathered, world, dA, dB, n_g, m, n);
-  return cudaGetLastError() == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(cudaGetLastError(), "merge_ranks launch");
 }
 
 int32_t grkan_forward_path(const void* x, const void* y, int64_t B, int64_t N, int64_t d,
@@ -416,12 +435,11 @@ int32_t grkan_backward_path(const void* x, const void* dy, const void* dx, int64
 grkan_status_t grkan_device_error(uint32_t* code, void* stream) {
   if (!code) return GRKAN_ERR_NULL;
   cudaStream_t st = (cudaStream_t)stream;
-  if (grk::read_device_error(code, st) != cudaSuccess) return GRKAN_ERR_CUDA;
-  return GRKAN_OK;
+  return cuda_status(grk::read_device_error(code, st), "grkan_device_error");
 }
 
 grkan_status_t grkan_clear_device_error(void* stream) {
-  return grk::clear_device_error((cudaStream_t)stream) == cudaSuccess ? GRKAN_OK : GRKAN_ERR_CUDA;
+  return cuda_status(grk::clear_device_error((cudaStream_t)stream), "grkan_clear_device_error");
 }
 
 const char* grkan_status_string(grkan_status_t s) {
@@ -441,5 +459,7 @@ const char* grkan_status_string(grkan_status_t s) {
 }
 
 int32_t grkan_abi_version(void) { return GRKAN_ABI_VERSION; }
+
+const char* grkan_last_error(void) { return g_last_error; }
 
 }  // extern "C"

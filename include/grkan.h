@@ -164,6 +164,11 @@ GRKAN_API grkan_status_t grkan_clear_device_error(void* stream);
 /* Human-readable name of a status code (static string). */
 GRKAN_API const char* grkan_status_string(grkan_status_t status);
 
+/* Text of the last CUDA-level failure on the calling thread (the failing call
+ * and CUDA's message) behind a GRKAN_ERR_CUDA return; static storage, valid
+ * until the thread's next failing call. */
+GRKAN_API const char* grkan_last_error(void);
+
 /* GRKAN_ABI_VERSION of the built library. */
 GRKAN_API int32_t grkan_abi_version(void);
 
