@@ -605,16 +605,21 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 
 // --- host-side launchers ---------------------------------------------------------
 
-// Raise the kernel's dynamic shared-memory limit to the largest layout it can
-// need (set once per kernel and device; later calls only compare).
-template <class K>
-inline cudaError_t set_smem(K kernel, unsigned most) {
+// Raise a kernel's dynamic shared-memory limit to the largest layout it can
+// need. One cache per kernel instantiation (the instantiations share a
+// function-pointer type, so the cache is keyed on the template arguments);
+// set once per device.
+template <class IO, bool kBackward>
+inline cudaError_t ensure_smem(unsigned most) {
   static int done_for_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (done_for_device == dev) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+  if (kBackward)
+    e = cudaFuncSetAttribute(bwd_tma<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+  else
+    e = cudaFuncSetAttribute(fwd_tma<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
   if (e == cudaSuccess) done_for_device = dev;
   return e;
 }
@@ -630,10 +635,10 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   if (grid > items) grid = items;
   cudaError_t e;
   if (bf16) {
-    if ((e = set_smem(fwd_tma<IoBF16>, most)) != cudaSuccess) return e;
+    if ((e = (ensure_smem<IoBF16, false>(most))) != cudaSuccess) return e;
     fwd_tma<IoBF16><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, my, a, b, g);
   } else {
-    if ((e = set_smem(fwd_tma<IoF32>, most)) != cudaSuccess) return e;
+    if ((e = (ensure_smem<IoF32, false>(most))) != cudaSuccess) return e;
     fwd_tma<IoF32><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, my, a, b, g);
   }
   return cudaGetLastError();
@@ -650,10 +655,10 @@ inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   if (grid > units) grid = units;
   cudaError_t e;
   if (bf16) {
-    if ((e = set_smem(bwd_tma<IoBF16>, most)) != cudaSuccess) return e;
+    if ((e = (ensure_smem<IoBF16, true>(most))) != cudaSuccess) return e;
     bwd_tma<IoBF16><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, mdy, mdx, a, b, ws, g);
   } else {
-    if ((e = set_smem(bwd_tma<IoF32>, most)) != cudaSuccess) return e;
+    if ((e = (ensure_smem<IoF32, true>(most))) != cudaSuccess) return e;
     bwd_tma<IoF32><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, mdy, mdx, a, b, ws, g);
   }
   return cudaGetLastError();

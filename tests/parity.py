@@ -7,9 +7,15 @@ Tolerances (the stated targets, made precise):
           Where the sign of Q(x) is undecidable in float32
           (|Q| < AMB_REL * sum_j |b_j||x|^j), dx may take the value of any of
           the three branches s = -1, 0, +1: each is a correct float32 result.
-  dA, dB  |gpu - ref| <= 1e-4 * |ref| + allowance, where the allowance is the
-          most that the undecidable signs can move dB (2 |dy y x^j / D| summed
-          over those elements; zero for dA, which does not depend on s).
+  dA, dB  |gpu - ref| <= 1e-4 * |ref| + 1e-5 * S_abs / sqrt(n_terms) + allowance.
+          S_abs = sum of |term| and n_terms = elements per group, so
+          S_abs / sqrt(n_terms) is the typical size of a sum of that many
+          random-sign terms: the floor is a tenth of the relative budget at
+          that size, and keeps a sum that cancels far below its own float32
+          rounding noise (|ref| << S_abs) from being graded on relative error.
+          The allowance is the most that the undecidable signs can move dB
+          (2 |dy y x^j / D| summed over those elements; zero for dA, which does
+          not depend on s).
 """
 import numpy as np
 import torch
@@ -61,18 +67,21 @@ def check_dx(got, ref, ex, rtol, what="dx"):
     return int(amb.sum())
 
 
-def check_coef(dA, dB, ref, rtol=RTOL_COEF, what=""):
-    """dA, dB: numpy float32/float64 arrays from the GPU; ref: oracle.coef_grads dict."""
+def check_coef(dA, dB, ref, n_terms, rtol=RTOL_COEF, floor=1e-5, what=""):
+    """dA, dB: numpy arrays from the GPU; ref: oracle.coef_grads dict;
+    n_terms: elements summed per group (rows * d_g). Returns the largest plain
+    relative error (for information)."""
     dA = np.asarray(dA, np.float64)
     dB = np.asarray(dB, np.float64)
+    s = float(np.sqrt(max(n_terms, 1)))
     eA = np.abs(dA - ref["dA"])
     eB = np.abs(dB - ref["dB"])
-    okA = eA <= rtol * np.abs(ref["dA"])
-    okB = eB <= rtol * np.abs(ref["dB"]) + ref["amb_b"]
-    assert okA.all(), "%s dA: max rel err %.3g (%s)" % (
-        what, float(np.max(eA / np.maximum(np.abs(ref["dA"]), 1e-300))), np.argwhere(~okA)[:4])
-    assert okB.all(), "%s dB: max rel err %.3g (%s)" % (
-        what, float(np.max(eB / np.maximum(np.abs(ref["dB"]), 1e-300))), np.argwhere(~okB)[:4])
-    rel = max(float(np.max(eA / np.maximum(np.abs(ref["dA"]), 1e-300), initial=0)),
-              float(np.max(eB / np.maximum(np.abs(ref["dB"]), 1e-300), initial=0)))
-    return rel
+    okA = eA <= rtol * np.abs(ref["dA"]) + floor * ref["sabs_a"] / s
+    okB = eB <= rtol * np.abs(ref["dB"]) + floor * ref["sabs_b"] / s + ref["amb_b"]
+    relA = eA / np.maximum(np.abs(ref["dA"]), 1e-300)
+    relB = eB / np.maximum(np.abs(ref["dB"]), 1e-300)
+    assert okA.all(), "%s dA: max rel err %.3g at %s" % (what, float(relA.max()),
+                                                         np.argwhere(~okA)[:4].tolist())
+    assert okB.all(), "%s dB: max rel err %.3g at %s" % (what, float(relB.max()),
+                                                         np.argwhere(~okB)[:4].tolist())
+    return max(float(relA.max(initial=0)), float(relB.max(initial=0)))
