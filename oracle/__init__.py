@@ -60,7 +60,7 @@ class Oracle:
         lib.gro_backward_elem.argtypes = [P, P, I, I64, I64, I, I, I, P, P, P, I64, P, P, P, P, P]
         lib.gro_backward_elem.restype = I
         lib.gro_coef_grads.argtypes = [P, P, I, I64, I64, I, I, I, P, P, ctypes.c_double, P, P, P,
-                                       P, P, P, I]
+                                       P, P, P, P, P, I]
         lib.gro_coef_grads.restype = I
         lib.gro_max_threads.restype = I
         self.lib = lib
@@ -129,8 +129,8 @@ class Oracle:
             "q": q.reshape(shape), "kappa_q": kq.reshape(shape)}
 
     def coef_grads(self, x, dy, a, b, n_g, amb_rel=AMB_REL, nthreads=0):
-        """dict with dA (n_g, m+1), dB (n_g, n), sabs_a, sabs_b, amb_b (float64)
-        and amb_count."""
+        """dict with dA (n_g, m+1), dB (n_g, n), sabs_a, sabs_b (sums of |term|),
+        c2_a, c2_b (conditioned sums of squares), amb_b (float64) and amb_count."""
         x, dtype, rows, d, a, b, m, n = self._prep(x, a, b, n_g)
         dy = np.ascontiguousarray(dy)
         assert dy.dtype == x.dtype and dy.shape == x.shape
@@ -138,16 +138,19 @@ class Oracle:
         dB = np.empty((n_g, n), np.float64)
         sa = np.empty_like(dA)
         sb = np.empty_like(dB)
+        ca = np.empty_like(dA)
+        cb = np.empty_like(dB)
         ab = np.empty_like(dB)
         cnt = ctypes.c_int64(0)
         rc = self.lib.gro_coef_grads(x.ctypes.data, dy.ctypes.data, dtype, rows, d, n_g, m, n,
                                      a.ctypes.data, b.ctypes.data, float(amb_rel), dA.ctypes.data,
                                      dB.ctypes.data, sa.ctypes.data, sb.ctypes.data,
-                                     ab.ctypes.data, ctypes.addressof(cnt), int(nthreads))
+                                     ca.ctypes.data, cb.ctypes.data, ab.ctypes.data,
+                                     ctypes.addressof(cnt), int(nthreads))
         if rc:
             raise ValueError("gro_coef_grads returned %d" % rc)
-        return {"dA": dA, "dB": dB, "sabs_a": sa, "sabs_b": sb, "amb_b": ab,
-                "amb_count": int(cnt.value)}
+        return {"dA": dA, "dB": dB, "sabs_a": sa, "sabs_b": sb, "c2_a": ca, "c2_b": cb,
+                "amb_b": ab, "amb_count": int(cnt.value)}
 
     def max_threads(self) -> int:
         return int(self.lib.gro_max_threads())

@@ -168,10 +168,19 @@ int gro_backward_elem(const void* x, const void* dy, int dtype, int64_t rows, in
   return 0;
 }
 
+static double kappa_p_at(double x, const double* a, int m) {
+  double ax = fabs(x), sa = 0.0, xi = 1.0;
+  for (int i = 0; i <= m; ++i) {
+    sa += fabs(a[i]) * xi;
+    xi *= ax;
+  }
+  return sa;
+}
+
 int gro_coef_grads(const void* x, const void* dy, int dtype, int64_t rows, int64_t d, int n_g,
                    int m, int n, const double* a, const double* b, double amb_rel, double* dA,
-                   double* dB, double* sabs_a, double* sabs_b, double* amb_b, int64_t* amb_count,
-                   int nthreads) {
+                   double* dB, double* sabs_a, double* sabs_b, double* c2_a, double* c2_b,
+                   double* amb_b, int64_t* amb_count, int nthreads) {
   int rc = check_args(rows, d, n_g, m, n, dtype);
   if (rc) return rc;
   if (!dA || (n > 0 && !dB)) return 4;
@@ -180,13 +189,14 @@ int gro_coef_grads(const void* x, const void* dy, int dtype, int64_t rows, int64
   const int ka = m + 1;
   const int kb = n;
   const int64_t dg = d / n_g;
-  /* Per chunk: dA, dB, |dA|, |dB|, amb_b, each n_g * (m+1+n) doubles, plus a count. */
+  /* Per chunk: sums, sums of |term|, conditioned sums of squares and the dB
+   * ambiguity allowance, each n_g * (m+1+n) doubles, plus a count. */
   const int64_t width = (int64_t)n_g * (ka + kb);
   const int64_t nchunks = (rows + GRO_CHUNK_ROWS - 1) / GRO_CHUNK_ROWS;
   double* part = NULL;
   int64_t* part_cnt = NULL;
   if (nchunks > 0) {
-    part = (double*)calloc((size_t)(nchunks * width * 3), sizeof(double));
+    part = (double*)calloc((size_t)(nchunks * width * 4), sizeof(double));
     part_cnt = (int64_t*)calloc((size_t)nchunks, sizeof(int64_t));
     if (!part || !part_cnt) {
       free(part);
@@ -199,9 +209,10 @@ int gro_coef_grads(const void* x, const void* dy, int dtype, int64_t rows, int64
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
 #endif
   for (int64_t c = 0; c < nchunks; ++c) {
-    double* sum = part + c * width * 3; /* [g][k] sums, k < ka: a_k, k >= ka: b_{k-ka+1} */
+    double* sum = part + c * width * 4; /* [g][k] sums, k < ka: a_k, k >= ka: b_{k-ka+1} */
     double* sab = sum + width;          /* sums of |term| */
     double* amb = sab + width;          /* ambiguity allowance for dB */
+    double* csq = amb + width;          /* conditioned sums of squares */
     int64_t r0 = c * GRO_CHUNK_ROWS;
     int64_t r1 = r0 + GRO_CHUNK_ROWS < rows ? r0 + GRO_CHUNK_ROWS : rows;
     for (int64_t r = r0; r < r1; ++r) {
@@ -217,20 +228,28 @@ int gro_coef_grads(const void* x, const void* dy, int dtype, int64_t rows, int64
         double* srow = sum + (int64_t)g * (ka + kb);
         double* arow = sab + (int64_t)g * (ka + kb);
         double* mrow = amb + (int64_t)g * (ka + kb);
+        double* qrow = csq + (int64_t)g * (ka + kb);
+        const double kq = kappa_q_at(xv, gb, n);
+        const double kp = kappa_p_at(xv, ga, m);
         double xi = 1.0;
         for (int i = 0; i <= m; ++i) {
           double term = gv * xi / p.D;
           srow[i] += term;
           arow[i] += fabs(term);
+          double w = fabs(term) * (1.0 + kq / p.D);
+          qrow[i] += w * w;
           xi *= xv;
         }
-        int ambiguous = fabs(p.Q) < amb_rel * kappa_q_at(xv, gb, n);
+        int ambiguous = fabs(p.Q) < amb_rel * kq;
         if (ambiguous) part_cnt[c] += 1;
         xi = xv;
         for (int j = 1; j <= n; ++j) {
           double term = -gv * p.y * p.s * xi / p.D;
           srow[ka + j - 1] += term;
           arow[ka + j - 1] += fabs(term);
+          double w = fabs(term) +
+                     fabs(gv * xi / (p.D * p.D)) * (kp + 2.0 * fabs(p.P) * kq / p.D);
+          qrow[ka + j - 1] += w * w;
           if (ambiguous) mrow[ka + j - 1] += 2.0 * fabs(gv * p.y * xi / p.D);
           xi *= xv;
         }
@@ -241,28 +260,33 @@ int gro_coef_grads(const void* x, const void* dy, int dtype, int64_t rows, int64
     for (int i = 0; i < ka; ++i) {
       dA[g * ka + i] = 0.0;
       if (sabs_a) sabs_a[g * ka + i] = 0.0;
+      if (c2_a) c2_a[g * ka + i] = 0.0;
     }
     for (int j = 0; j < kb; ++j) {
       dB[g * kb + j] = 0.0;
       if (sabs_b) sabs_b[g * kb + j] = 0.0;
+      if (c2_b) c2_b[g * kb + j] = 0.0;
       if (amb_b) amb_b[g * kb + j] = 0.0;
     }
   }
   int64_t namb = 0;
   for (int64_t c = 0; c < nchunks; ++c) {
-    const double* sum = part + c * width * 3;
+    const double* sum = part + c * width * 4;
     const double* sab = sum + width;
     const double* amb = sab + width;
+    const double* csq = amb + width;
     namb += part_cnt[c];
     for (int g = 0; g < n_g; ++g) {
       const int64_t o = (int64_t)g * (ka + kb);
       for (int i = 0; i < ka; ++i) {
         dA[g * ka + i] += sum[o + i];
         if (sabs_a) sabs_a[g * ka + i] += sab[o + i];
+        if (c2_a) c2_a[g * ka + i] += csq[o + i];
       }
       for (int j = 0; j < kb; ++j) {
         dB[g * kb + j] += sum[o + ka + j];
         if (sabs_b) sabs_b[g * kb + j] += sab[o + ka + j];
+        if (c2_b) c2_b[g * kb + j] += csq[o + ka + j];
         if (amb_b) amb_b[g * kb + j] += amb[o + ka + j];
       }
     }

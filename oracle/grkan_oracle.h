@@ -70,6 +70,16 @@ int gro_backward_elem(const void* x, const void* dy, int dtype, int64_t rows, in
 /* Coefficient gradients over all rows:
  *   dA[n_g][m+1], dB[n_g][n]           the sums
  *   sabs_a, sabs_b (nullable)          sums of |term| (condition scale)
+ *   c2_a, c2_b (nullable)              sums of (|term| (1 + c))^2, c the
+ *                                      term's sensitivity to float32 rounding
+ *                                      of the polynomials it depends on:
+ *                                      c = kappa_q / D for a dA term
+ *                                      (kappa_q = sum_j |b_j||x|^j), and
+ *                                      |term| (1 + c) = |term| + |g x^j / D^2|
+ *                                      (kappa_p + 2 |P| kappa_q / D) for a dB
+ *                                      term (kappa_p = sum_i |a_i||x|^i); the
+ *                                      square root is the size of the float32
+ *                                      rounding noise of the sum
  *   amb_b (nullable)                   sum over elements whose sign decision is
  *                                      ambiguous (|Q| < amb_rel * kappa_q) of
  *                                      2 |g y x^j / D|: the most a flipped sign
@@ -78,8 +88,8 @@ int gro_backward_elem(const void* x, const void* dy, int dtype, int64_t rows, in
  * nthreads <= 0 uses every available thread. */
 int gro_coef_grads(const void* x, const void* dy, int dtype, int64_t rows, int64_t d, int n_g,
                    int m, int n, const double* a, const double* b, double amb_rel, double* dA,
-                   double* dB, double* sabs_a, double* sabs_b, double* amb_b, int64_t* amb_count,
-                   int nthreads);
+                   double* dB, double* sabs_a, double* sabs_b, double* c2_a, double* c2_b,
+                   double* amb_b, int64_t* amb_count, int nthreads);
 
 int gro_max_threads(void);
 

@@ -341,6 +341,30 @@ def pin_ambiguity(orc):
     _close(g["amb_b"][0], want, 1e-15, 0, "ambiguity allowance")
 
 
+def pin_noise_scales(orc):
+    """c2 (the conditioned sums of squares used as the float32 noise scale of
+    dA / dB): with b = 0 the denominator is exactly 1 and Q is exactly 0, so
+    c2_a = sum (dy x^i)^2 and c2_b = sum (|dy x^j| sum_i |a_i||x|^i)^2; in general
+    c2 >= sabs^2 / n_terms (Cauchy-Schwarz, the weights being >= 1)."""
+    rng = np.random.default_rng(14)
+    rows, d, n_g, m, n = 9, 12, 3, 5, 4
+    x, dy, a, b = _rand_case(rng, rows, d, n_g, m, n)
+    dg = d // n_g
+    g0 = orc.coef_grads(x, dy, a, np.zeros_like(b), n_g)
+    xs = x.astype(np.float64).reshape(rows, n_g, dg)
+    gs = dy.astype(np.float64).reshape(rows, n_g, dg)
+    kp = sum(np.abs(a.astype(np.float64))[None, :, i, None] * np.abs(xs) ** i for i in range(m + 1))
+    for i in range(m + 1):
+        _close(g0["c2_a"][:, i], ((gs * xs ** i) ** 2).sum(axis=(0, 2)), 1e-13, 0, "c2_a b=0")
+    for j in range(1, n + 1):
+        _close(g0["c2_b"][:, j - 1], ((np.abs(gs * xs ** j) * kp) ** 2).sum(axis=(0, 2)), 1e-13,
+               0, "c2_b b=0")
+    g = orc.coef_grads(x, dy, a, b, n_g)
+    nt = rows * dg
+    assert np.all(g["c2_a"] >= g["sabs_a"] ** 2 / nt * (1 - 1e-12))
+    assert np.all(g["c2_b"] >= g["sabs_b"] ** 2 / nt * (1 - 1e-12))
+
+
 ALL_PINS = [pin_identity, pin_polynomial_b0, pin_dyadic_exact, pin_x_zero, pin_bf16_widening,
             pin_fd_dx, pin_fd_dA, pin_fd_dB, pin_autograd, pin_linearity, pin_group_relabel,
-            pin_thread_invariance, pin_sampled_and_extras, pin_ambiguity]
+            pin_thread_invariance, pin_sampled_and_extras, pin_ambiguity, pin_noise_scales]

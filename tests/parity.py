@@ -7,12 +7,18 @@ Tolerances (the stated targets, made precise):
           Where the sign of Q(x) is undecidable in float32
           (|Q| < AMB_REL * sum_j |b_j||x|^j), dx may take the value of any of
           the three branches s = -1, 0, +1: each is a correct float32 result.
-  dA, dB  |gpu - ref| <= 1e-4 * |ref| + 1e-5 * S_abs / sqrt(n_terms) + allowance.
-          S_abs = sum of |term| and n_terms = elements per group, so
-          S_abs / sqrt(n_terms) is the typical size of a sum of that many
-          random-sign terms: the floor is a tenth of the relative budget at
-          that size, and keeps a sum that cancels far below its own float32
-          rounding noise (|ref| << S_abs) from being graded on relative error.
+  dA, dB  |gpu - ref| <= 1e-4 * |ref| + 2e-6 * sqrt(c2) + allowance.
+          c2 (from the oracle) is the sum over the group's elements of
+          (|term| (1 + c))^2, c the term's sensitivity to float32 rounding of
+          P and Q. Random per-term and per-addition rounding errors add in
+          quadrature, so the float32 noise of the sum is a few u * sqrt(c2)
+          (u = 2^-24 = 6e-8; the per-addition part also grows with the square
+          root of the summation depth, ~10 here): 2e-6 = 32 u leaves a margin
+          of 5 to 20 above it. For random-sign, light-tailed terms sqrt(c2) ~
+          |ref|, so the floor is 2% of the relative budget; it matters only for
+          a sum that cancels far below its own rounding noise
+          (|ref| << sum |term|) or one dominated by a few ill-conditioned,
+          heavy-tailed terms, where float32 terms cannot reach 1e-4 relative.
           The allowance is the most that the undecidable signs can move dB
           (2 |dy y x^j / D| summed over those elements; zero for dA, which does
           not depend on s).
@@ -67,17 +73,15 @@ def check_dx(got, ref, ex, rtol, what="dx"):
     return int(amb.sum())
 
 
-def check_coef(dA, dB, ref, n_terms, rtol=RTOL_COEF, floor=1e-5, what=""):
-    """dA, dB: numpy arrays from the GPU; ref: oracle.coef_grads dict;
-    n_terms: elements summed per group (rows * d_g). Returns the largest plain
-    relative error (for information)."""
+def check_coef(dA, dB, ref, rtol=RTOL_COEF, floor=2e-6, what=""):
+    """dA, dB: numpy arrays from the GPU; ref: oracle.coef_grads dict. Returns
+    the largest plain relative error (for information)."""
     dA = np.asarray(dA, np.float64)
     dB = np.asarray(dB, np.float64)
-    s = float(np.sqrt(max(n_terms, 1)))
     eA = np.abs(dA - ref["dA"])
     eB = np.abs(dB - ref["dB"])
-    okA = eA <= rtol * np.abs(ref["dA"]) + floor * ref["sabs_a"] / s
-    okB = eB <= rtol * np.abs(ref["dB"]) + floor * ref["sabs_b"] / s + ref["amb_b"]
+    okA = eA <= rtol * np.abs(ref["dA"]) + floor * np.sqrt(ref["c2_a"])
+    okB = eB <= rtol * np.abs(ref["dB"]) + floor * np.sqrt(ref["c2_b"]) + ref["amb_b"]
     relA = eA / np.maximum(np.abs(ref["dA"]), 1e-300)
     relB = eB / np.maximum(np.abs(ref["dB"]), 1e-300)
     assert okA.all(), "%s dA: max rel err %.3g at %s" % (what, float(relA.max()),

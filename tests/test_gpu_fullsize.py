@@ -53,8 +53,7 @@ def test_fullsize(name, n_g):
     check_dx(dx_s, dx_ref, ex, rtol, "%s dx" % w.name)
 
     g_ref = oracle.coef_grads(x, dy, a, b, w.n_g)
-    rel = check_coef(dA.cpu().numpy(), dB.cpu().numpy(), g_ref, w.rows * (w.d // w.n_g),
-                     what=w.name)
+    rel = check_coef(dA.cpu().numpy(), dB.cpu().numpy(), g_ref, what=w.name)
     print("%s: max plain relative error of dA/dB %.3g, ambiguous signs %d" % (
         w.name, rel, g_ref["amb_count"]))
 

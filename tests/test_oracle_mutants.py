@@ -40,6 +40,9 @@ MUTANTS = [
     ("last reduction chunk dropped", "  for (int64_t c = 0; c < nchunks; ++c) {\n    const double* sum",
      "  for (int64_t c = 0; c + 1 < nchunks; ++c) {\n    const double* sum", 0),
     ("bf16 widened from the wrong half", "<< 16;", "<< 15;", 0),
+    ("noise scale not squared", "qrow[i] += w * w;", "qrow[i] += w;", 0),
+    ("dB noise scale drops kappa_p", "(kp + 2.0 * fabs(p.P) * kq / p.D)", "(2.0 * fabs(p.P) * kq / p.D)",
+     0),
     ("forward groups interleaved", "int g = (int)((e % d) / dg);",
      "int g = (int)((e % d) % n_g);", 0),
 ]
