@@ -38,6 +38,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="kat_b", choices=list(synth.WORKLOADS))
     ap.add_argument("--ng", type=int, default=None, help="groups for the stress workload")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="use only the first ROWS rows of the workload (profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
@@ -177,6 +179,10 @@ def run_reference(args, w):
 def main():
     args = parse()
     w = synth.workload(args.config, n_g=args.ng)
+    if args.rows is not None:
+        w = w.with_rows(args.rows)
+        w.B, w.N = args.rows, 1
+        w.rows_override = None
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -291,7 +297,7 @@ def main():
         dA_h.copy_(dA, non_blocking=True)
         dB_h.copy_(dB, non_blocking=True)
 
-    for _ in range(2):
+    for _ in range(min(2, args.e2e_steps)):
         e2e_step()
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -303,7 +309,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / max(args.e2e_steps, 1)
     if world > 1:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

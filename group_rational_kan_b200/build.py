@@ -41,10 +41,12 @@ def needs_build():
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def command(out=LIB, verbose=False):
+def command(out=LIB, verbose=False, defines=()):
+    """nvcc command line; ``defines`` are extra -D settings of the launch-shape
+    knobs in csrc/grkan_tma.cuh (GRK_CONSUMER_WARPS, GRK_CTAS_PER_SM, ...)."""
     cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
            "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
-           "-DGRKAN_BUILD_SHARED", "-o", out, *SOURCES]
+           *["-D" + d for d in defines], "-o", out, *SOURCES]
     if verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     return cmd

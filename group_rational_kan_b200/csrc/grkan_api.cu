@@ -36,7 +36,7 @@ grkan_status_t cuda_status(cudaError_t e, const char* where) {
 // tensor); a unit (row tile x group) is kChunksPerUnit chunks. The partition
 // depends only on the shape, never on the device, so the float32 partials --
 // and therefore dA and dB -- are the same bits on every run.
-constexpr long long kChunkBytes = 12288;
+constexpr long long kChunkBytes = GRK_CHUNK_BYTES;
 constexpr int kChunksPerUnit = 4;
 constexpr int kMaxBoxRows = 256;
 

@@ -44,14 +44,37 @@ struct TmaGeom {
   int m, n;             // degrees
 };
 
-constexpr int kConsumerWarps = 8;
+// Launch shape (compile-time; the defaults are the tuned configuration).
+#ifndef GRK_CONSUMER_WARPS
+#define GRK_CONSUMER_WARPS 8
+#endif
+#ifndef GRK_CTAS_PER_SM
+#define GRK_CTAS_PER_SM 2
+#endif
+#ifndef GRK_FWD_STAGES
+#define GRK_FWD_STAGES 8
+#endif
+#ifndef GRK_BWD_STAGES
+#define GRK_BWD_STAGES 4
+#endif
+#ifndef GRK_CHUNK_BYTES
+#define GRK_CHUNK_BYTES 12288
+#endif
+// registers per thread so that GRK_CTAS_PER_SM CTAs fit the 64K register file
+#define GRK_MAXNREG                                                                        \
+  ((65536 / ((GRK_CONSUMER_WARPS + 1) * 32 * GRK_CTAS_PER_SM)) / 8 * 8 > 255               \
+       ? 255                                                                               \
+       : (65536 / ((GRK_CONSUMER_WARPS + 1) * 32 * GRK_CTAS_PER_SM)) / 8 * 8)
+
+constexpr int kConsumerWarps = GRK_CONSUMER_WARPS;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kTmaThreads = kConsumers + 32;
-constexpr int kFwdStages = 8;
-constexpr int kBwdStages = 4;
-constexpr unsigned kMaxChunkBytes = 12288;
-constexpr int kMaxVecPerThread = (int)(kMaxChunkBytes / 16 / kConsumers);  // 3
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;             // 2 s
+constexpr int kCtasPerSm = GRK_CTAS_PER_SM;
+constexpr int kFwdStages = GRK_FWD_STAGES;
+constexpr int kBwdStages = GRK_BWD_STAGES;
+constexpr unsigned kMaxChunkBytes = GRK_CHUNK_BYTES;
+constexpr int kMaxVecPerThread = (int)((kMaxChunkBytes / 16 + kConsumers - 1) / kConsumers);
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 
 // Error codes written to g_grkan_device_error (bit-or).
 constexpr unsigned kErrFullWait = 1u;
@@ -271,7 +294,7 @@ __device__ __forceinline__ int unit_chunks(const TmaGeom& g, long long tile) {
 // taken by CTA i as w = i, i + grid, ...
 
 template <class IO>
-__global__ void __maxnreg__(112)
+__global__ void __maxnreg__(GRK_MAXNREG)
 fwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap my,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -410,7 +433,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 // of unit (tile, g), coefficient k go to ws[(g * 10 + k) * T + tile].
 
 template <class IO>
-__global__ void __maxnreg__(112)
+__global__ void __maxnreg__(GRK_MAXNREG)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
         const __grid_constant__ CUtensorMap mdx, const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
@@ -631,7 +654,7 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   const unsigned most = Layout(kMaxChunkBytes, 1, kFwdStages, false).total;
   if (L.total > most) return cudaErrorInvalidValue;
   const long long items = ((g.rows + g.SC - 1) / g.SC) * g.n_g;
-  long long grid = 2LL * sms;
+  long long grid = (long long)kCtasPerSm * sms;
   if (grid > items) grid = items;
   cudaError_t e;
   if (bf16) {
@@ -651,7 +674,7 @@ inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   const unsigned most = Layout(kMaxChunkBytes, 2, kBwdStages, true).total;
   if (L.total > most) return cudaErrorInvalidValue;
   const long long units = g.T * g.n_g;
-  long long grid = 2LL * sms;
+  long long grid = (long long)kCtasPerSm * sms;
   if (grid > units) grid = units;
   cudaError_t e;
   if (bf16) {
