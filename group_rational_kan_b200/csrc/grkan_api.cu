@@ -222,6 +222,7 @@ bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
 grk::TmaGeom make_geom(const Plan& p, int bw) {
   grk::TmaGeom g;
   g.rows = p.rows;
+  g.d = p.d;
   g.dg = (int)p.dg;
   g.n_g = p.n_g;
   g.SC = p.SC;
@@ -250,21 +251,20 @@ int sm_count() {
 grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float* a,
                               const float* b, cudaStream_t st) {
   const int bw = tma_box_width(p);
-  CUtensorMap mx, my;
-  if (!make_map(&mx, x, p, bw) || !make_map(&my, y, p, bw)) return GRKAN_ERR_CUDA;
+  CUtensorMap mx;
+  if (!make_map(&mx, x, p, bw)) return GRKAN_ERR_CUDA;
   const grk::TmaGeom geom = make_geom(p, bw);
-  cudaError_t e = grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, my, a, b, sm_count(), st);
+  cudaError_t e = grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, y, a, b, sm_count(), st);
   return cuda_status(e, "forward (TMA) launch");
 }
 
 grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx,
                               const float* a, const float* b, float* ws, cudaStream_t st) {
   const int bw = tma_box_width(p);
-  CUtensorMap mx, mdy, mdx;
-  if (!make_map(&mx, x, p, bw) || !make_map(&mdy, dy, p, bw) || !make_map(&mdx, dx, p, bw))
-    return GRKAN_ERR_CUDA;
+  CUtensorMap mx, mdy;
+  if (!make_map(&mx, x, p, bw) || !make_map(&mdy, dy, p, bw)) return GRKAN_ERR_CUDA;
   const grk::TmaGeom geom = make_geom(p, bw);
-  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, mdx, a, b, ws,
+  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, dx, a, b, ws,
                                       sm_count(), st);
   return cuda_status(e, "backward (TMA) launch");
 }

@@ -2,22 +2,21 @@
 //
 // Work decomposition: (row tile x group) units as in the FlashKAT backward
 // ("FlashKAT ...", paper notes, section "3. FlashKAT kernel restructuring
-// (Algorithm 2)"), realised as a persistent grid of two CTAs per SM that walk
-// the unit list in a fixed stride. Each unit is split into chunks of SC rows x
-// d_g channels (about 12 KiB per tensor) that stream through a ring of shared-
-// memory stages:
-//   warp 0 (one elected lane) : stages the group's coefficients into the
-//       stage's header, issues 2-D TMA tile loads of x (and dy) into the stage,
-//       and once the consumers release a stage, a 2-D TMA tile store of the
-//       result (y or dx) the consumers wrote in place;
-//   warps 1..8 (consumers)     : evaluate the rational function on pairs of
-//       elements with packed float32x2 arithmetic and, in the backward, keep
-//       the ten coefficient-gradient sums in registers.
-// At the end of a backward unit the consumers fold their sums through shared
-// memory and warp shuffles, in a fixed order, into one float32 partial per
-// (unit, coefficient) in the workspace -- no atomics anywhere
-// (section "3. ...": accumulate inside the block, one global write per block).
-//
+// (Algorithm 2)"), realised as a persistent grid of one 16-warp CTA per SM that
+// walks the unit list in a fixed stride. A unit is split into chunks of SC rows
+// x d_g channels (24 KiB of one tensor) that stream through a ring of shared-
+// memory stages filled by 2-D TMA tile loads:
+//   - thread 0 also acts as the issuer: it stages the group's coefficients in
+//     the stage header and issues the loads, keeping the ring full by refilling
+//     the stage of chunk q-1 (once every warp has read it) when it starts q;
+//   - every warp reads its vectors of the chunk into registers, releases the
+//     stage, evaluates the rational function on pairs of elements with packed
+//     float32x2 arithmetic, and writes y or dx with 16-byte global stores;
+//   - the backward keeps the ten coefficient-gradient sums in registers; at the
+//     end of a unit they are folded in a fixed order through shared memory and
+//     warp shuffles into one float32 partial per (unit, coefficient) in the
+//     workspace -- no atomics (section "3. ...": accumulate inside the block,
+//     one global write per block).
 // Every wait is bounded: a wait that runs out records a code in
 // g_grkan_device_error and the kernel winds down instead of hanging.
 #pragma once
@@ -34,6 +33,7 @@ namespace grk {
 struct TmaGeom {
   long long rows;       // B * N
   long long T;          // row tiles
+  long long d;          // channels (row length)
   int dg;               // channels per group
   int n_g;              // groups
   int SC;               // rows per chunk (TMA box height)
@@ -45,11 +45,8 @@ struct TmaGeom {
 };
 
 // Launch shape (compile-time; the defaults are the tuned configuration).
-#ifndef GRK_CONSUMER_WARPS
-#define GRK_CONSUMER_WARPS 8
-#endif
-#ifndef GRK_CTAS_PER_SM
-#define GRK_CTAS_PER_SM 2
+#ifndef GRK_WARPS
+#define GRK_WARPS 16
 #endif
 #ifndef GRK_FWD_STAGES
 #define GRK_FWD_STAGES 8
@@ -58,23 +55,16 @@ struct TmaGeom {
 #define GRK_BWD_STAGES 4
 #endif
 #ifndef GRK_CHUNK_BYTES
-#define GRK_CHUNK_BYTES 12288
+#define GRK_CHUNK_BYTES 24576
 #endif
-// registers per thread so that GRK_CTAS_PER_SM CTAs fit the 64K register file
-#define GRK_MAXNREG                                                                        \
-  ((65536 / ((GRK_CONSUMER_WARPS + 1) * 32 * GRK_CTAS_PER_SM)) / 8 * 8 > 255               \
-       ? 255                                                                               \
-       : (65536 / ((GRK_CONSUMER_WARPS + 1) * 32 * GRK_CTAS_PER_SM)) / 8 * 8)
 
-constexpr int kConsumerWarps = GRK_CONSUMER_WARPS;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kTmaThreads = kConsumers + 32;
-constexpr int kCtasPerSm = GRK_CTAS_PER_SM;
+constexpr int kWarps = GRK_WARPS;
+constexpr int kThreads = kWarps * 32;
 constexpr int kFwdStages = GRK_FWD_STAGES;
 constexpr int kBwdStages = GRK_BWD_STAGES;
 constexpr unsigned kMaxChunkBytes = GRK_CHUNK_BYTES;
-constexpr int kMaxVecPerThread = (int)((kMaxChunkBytes / 16 + kConsumers - 1) / kConsumers);
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+constexpr int kVec = (int)((kMaxChunkBytes / 16 + kThreads - 1) / kThreads);  // vectors/thread
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;                 // 2 s
 
 // Error codes written to g_grkan_device_error (bit-or).
 constexpr unsigned kErrFullWait = 1u;
@@ -142,22 +132,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1, uint32_t src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::
-                   "l"(reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(src)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -267,7 +241,7 @@ __host__ __device__ constexpr unsigned round_up(unsigned v, unsigned a) {
 }
 
 // [stages x tensors x chunk] [stages x header coef] [full bars] [empty bars]
-// [reduction bars] [reduction buffer]
+// [two reduction bars] [reduction buffer 10 x kThreads floats]
 struct Layout {
   unsigned stage_stride;  // bytes of one stage (all tensors)
   unsigned coef_off, bar_off, red_off, total;
@@ -277,7 +251,7 @@ struct Layout {
     coef_off = stage_stride * (unsigned)stages;
     bar_off = coef_off + (unsigned)(stages * kCoefSlot * 4);
     red_off = round_up(bar_off + (unsigned)(2 * stages + 2) * 8, 128);
-    total = red_off + (reduce ? (unsigned)(10 * kConsumers * 4) : 0u);
+    total = red_off + (reduce ? (unsigned)(10 * kThreads * 4) : 0u);
   }
 };
 
@@ -289,124 +263,138 @@ __device__ __forceinline__ int unit_chunks(const TmaGeom& g, long long tile) {
   return (int)((left + g.SC - 1) / g.SC);
 }
 
+// Where the vectors a thread owns in every chunk go in global memory. The
+// chunk is stored in shared memory as nbox boxes of SC rows x bw channels;
+// vector v (16 bytes) of the chunk is box v / (SC*vpr), row (v % (SC*vpr)) /
+// vpr, vector column v % vpr. off = element offset from the chunk's origin
+// (first row, first channel of the group); row = row within the chunk, or a
+// huge value for a slot past the end of the chunk.
+template <class IO>
+struct VecMap {
+  long long off[kVec];
+  int row[kVec];
+  __device__ __forceinline__ void init(const TmaGeom& g, int tid) {
+    constexpr int ve = 16 / IO::kBytes;  // elements per vector
+    const int vpr = g.bw / ve;
+    const int vpb = vpr * g.SC;
+    const int nvec = (int)(g.chunk_bytes / 16);
+#pragma unroll
+    for (int it = 0; it < kVec; ++it) {
+      const int v = tid + it * kThreads;
+      if (v < nvec) {
+        const int bx = v / vpb;
+        const int rem = v - bx * vpb;
+        const int r = rem / vpr;
+        const int c = rem - r * vpr;
+        row[it] = r;
+        off[it] = (long long)r * g.d + (long long)bx * g.bw + (long long)c * ve;
+      } else {
+        row[it] = 0x3fffffff;
+        off[it] = 0;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ void store16(void* p, uint4 v) {
+  __stcs(reinterpret_cast<uint4*>(p), v);
+}
+
 // --- forward -----------------------------------------------------------------------
 // Work items are (row chunk, group) pairs, item w -> chunk w / n_g, group w % n_g,
 // taken by CTA i as w = i, i + grid, ...
 
 template <class IO>
-__global__ void __maxnreg__(GRK_MAXNREG)
-fwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap my,
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const Layout L(geom.chunk_bytes, 1, kFwdStages, false);
   float* coef = reinterpret_cast<float*>(smem + L.coef_off);
   const uint32_t full0 = smem_addr(smem + L.bar_off);
   const uint32_t empty0 = full0 + 8 * kFwdStages;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
   const long long row_chunks = (geom.rows + geom.SC - 1) / geom.SC;
   const long long items = row_chunks * geom.n_g;
   const int box_bytes = geom.SC * geom.bw * IO::kBytes;
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kConsumerWarps);
+      mbar_init(empty0 + 8 * s, kWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
+    prefetch_map(&mx);
   }
   __syncthreads();
 
-  if (warp == 0) {
-    if (lane != 0) return;
-    prefetch_map(&mx);
-    prefetch_map(&my);
-    bool ok = true;
-    long long q = 0;  // chunk sequence number in this CTA
-    for (long long w = blockIdx.x; w < items; w += gridDim.x, ++q) {
-      const int s = (int)(q % kFwdStages);
-      const uint32_t kq = (uint32_t)(q / kFwdStages);
-      const long long rc = w / geom.n_g;
-      const int g = (int)(w - rc * geom.n_g);
-      if (q >= kFwdStages) {
-        // stage s held item w - kFwdStages*grid: store its y once consumers are done
-        if (!mbar_wait(empty0 + 8 * s, (kq - 1) & 1)) { report(kErrEmptyWait); ok = false; break; }
-        const long long wp = w - (long long)kFwdStages * gridDim.x;
-        const long long rcp = wp / geom.n_g;
-        const int gp = (int)(wp - rcp * geom.n_g);
-        for (int bx = 0; bx < geom.nbox; ++bx)
-          tma_store_2d(&my, gp * geom.dg + bx * geom.bw, (int)(rcp * geom.SC),
-                       smem_addr(smem + s * L.stage_stride + bx * box_bytes));
-        bulk_commit();
-        bulk_wait_read_all();
-      }
-      float* cs = coef + s * kCoefSlot;
+  // issue cursor (thread 0): next item to load and its sequence number
+  long long iw = blockIdx.x, iq = 0;
+  auto issue = [&]() {
+    const int s = (int)(iq % kFwdStages);
+    const long long rc = iw / geom.n_g;
+    const int g = (int)(iw - rc * geom.n_g);
+    float* cs = coef + s * kCoefSlot;
 #pragma unroll
-      for (int i = 0; i < 6; ++i) cs[i] = __ldg(a + g * 6 + i);
+    for (int i = 0; i < 6; ++i) cs[i] = __ldg(a + g * 6 + i);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) cs[6 + j] = __ldg(b + g * 4 + j);
-      mbar_arrive_expect_tx(full0 + 8 * s, geom.chunk_bytes);
-      for (int bx = 0; bx < geom.nbox; ++bx)
-        tma_load_2d(smem_addr(smem + s * L.stage_stride + bx * box_bytes), &mx,
-                    g * geom.dg + bx * geom.bw, (int)(rc * geom.SC), full0 + 8 * s);
-    }
-    // drain: store the last stages
-    if (ok) {
-      const long long first = q > kFwdStages ? q - kFwdStages : 0;
-      for (long long j = first; j < q; ++j) {
-        const int s = (int)(j % kFwdStages);
-        const uint32_t kj = (uint32_t)(j / kFwdStages);
-        if (!mbar_wait(empty0 + 8 * s, kj & 1)) { report(kErrEmptyWait); ok = false; break; }
-        const long long wj = blockIdx.x + j * (long long)gridDim.x;
-        const long long rcj = wj / geom.n_g;
-        const int gj = (int)(wj - rcj * geom.n_g);
-        for (int bx = 0; bx < geom.nbox; ++bx)
-          tma_store_2d(&my, gj * geom.dg + bx * geom.bw, (int)(rcj * geom.SC),
-                       smem_addr(smem + s * L.stage_stride + bx * box_bytes));
-        bulk_commit();
-      }
-    }
-    if (!ok) {
-      // wind down: let every issued load land before the CTA's memory goes away
-      const long long first = q > kFwdStages ? q - kFwdStages : 0;
-      for (long long j = first; j < q; ++j) {
-        if (!mbar_wait(full0 + 8 * (int)(j % kFwdStages), (uint32_t)(j / kFwdStages) & 1)) {
-          report(kErrDrainWait);
-        }
-      }
-    }
-    bulk_wait_all();
-    return;
-  }
+    for (int j = 0; j < 4; ++j) cs[6 + j] = __ldg(b + g * 4 + j);
+    mbar_arrive_expect_tx(full0 + 8 * s, geom.chunk_bytes);
+    for (int bx = 0; bx < geom.nbox; ++bx)
+      tma_load_2d(smem_addr(smem + s * L.stage_stride + bx * box_bytes), &mx,
+                  g * geom.dg + bx * geom.bw, (int)(rc * geom.SC), full0 + 8 * s);
+    iw += gridDim.x;
+    ++iq;
+  };
+  if (tid == 0)
+    for (int s = 0; s < kFwdStages && iw < items; ++s) issue();
 
-  // consumers
-  const int ct = threadIdx.x - 32;
+  VecMap<IO> vm;
+  vm.init(geom, tid);
   const int nvec = (int)(geom.chunk_bytes / 16);
   Coef54 c;
   int cur_g = -1;
+  bool ok = true;
   long long q = 0;
   for (long long w = blockIdx.x; w < items; w += gridDim.x, ++q) {
     const int s = (int)(q % kFwdStages);
-    const uint32_t kq = (uint32_t)(q / kFwdStages);
+    if (tid == 0 && q >= 1 && iw < items) {
+      // refill the stage of chunk q-1 once every warp has read it
+      if (!mbar_wait(empty0 + 8 * (int)((q - 1) % kFwdStages),
+                     (uint32_t)((q - 1) / kFwdStages) & 1)) {
+        report(kErrEmptyWait);
+        ok = false;
+        break;
+      }
+      issue();
+    }
+    if (!mbar_wait(full0 + 8 * s, (uint32_t)(q / kFwdStages) & 1)) {
+      report(kErrFullWait);
+      ok = false;
+      break;
+    }
     const long long rc = w / geom.n_g;
     const int g = (int)(w - rc * geom.n_g);
-    if (!mbar_wait(full0 + 8 * s, kq & 1)) { report(kErrFullWait); return; }
     if (g != cur_g) {
       c.set(coef + s * kCoefSlot);
       cur_g = g;
     }
-    uint4* buf = reinterpret_cast<uint4*>(smem + s * L.stage_stride);
-    uint4 v[kMaxVecPerThread];
+    const uint4* buf = reinterpret_cast<const uint4*>(smem + s * L.stage_stride);
+    uint4 v[kVec];
 #pragma unroll
-    for (int it = 0; it < kMaxVecPerThread; ++it) {
-      const int vi = ct + it * kConsumers;
+    for (int it = 0; it < kVec; ++it) {
+      const int vi = tid + it * kThreads;
       if (vi < nvec) v[it] = buf[vi];
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    const long long row0 = rc * geom.SC;
+    typename IO::T* yo = y + row0 * geom.d + (long long)g * geom.dg;
 #pragma unroll
-    for (int it = 0; it < kMaxVecPerThread; ++it) {
-      const int vi = ct + it * kConsumers;
-      if (vi < nvec) {
+    for (int it = 0; it < kVec; ++it) {
+      if (row0 + vm.row[it] < geom.rows) {
         uint4 o;
         if constexpr (IO::kBytes == 2) {
           o.x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].x)));
@@ -414,160 +402,156 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
           o.z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].z)));
           o.w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].w)));
         } else {
-          const float2 p0 = fwd_pair(c, make_float2(__uint_as_float(v[it].x), __uint_as_float(v[it].y)));
-          const float2 p1 = fwd_pair(c, make_float2(__uint_as_float(v[it].z), __uint_as_float(v[it].w)));
+          const float2 p0 =
+              fwd_pair(c, make_float2(__uint_as_float(v[it].x), __uint_as_float(v[it].y)));
+          const float2 p1 =
+              fwd_pair(c, make_float2(__uint_as_float(v[it].z), __uint_as_float(v[it].w)));
           o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
                          __float_as_uint(p1.y));
         }
-        buf[vi] = o;
+        store16(yo + vm.off[it], o);
       }
     }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+  }
+  if (!ok && tid == 0) {
+    // wind down: let every issued load land before the CTA's memory goes away
+    for (long long j = q; j < iq; ++j)
+      if (!mbar_wait(full0 + 8 * (int)(j % kFwdStages), (uint32_t)(j / kFwdStages) & 1))
+        report(kErrDrainWait);
   }
 }
 
 // --- backward ------------------------------------------------------------------------
-// Units u = tile * n_g + g, taken by CTA i as u = i, i + grid, ...; partial sums
-// of unit (tile, g), coefficient k go to ws[(g * 10 + k) * T + tile].
+// Units u = tile * n_g + g, taken by CTA i as u = i, i + grid, ...; the partial
+// sum of unit (tile, g), coefficient k goes to ws[(g * 10 + k) * T + tile].
 
 template <class IO>
-__global__ void __maxnreg__(GRK_MAXNREG)
+__global__ void __launch_bounds__(kThreads, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
-        const __grid_constant__ CUtensorMap mdx, const float* __restrict__ a,
+        typename IO::T* __restrict__ dx, const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const Layout L(geom.chunk_bytes, 2, kBwdStages, true);
-  const unsigned cbytes = round_up(geom.chunk_bytes, 128);  // x at +0, dy / dx at +cbytes
+  const unsigned cbytes = round_up(geom.chunk_bytes, 128);  // x at +0, dy at +cbytes
   float* coef = reinterpret_cast<float*>(smem + L.coef_off);
   const uint32_t full0 = smem_addr(smem + L.bar_off);
   const uint32_t empty0 = full0 + 8 * kBwdStages;
   const uint32_t redbar = empty0 + 8 * kBwdStages;  // two: "written", "read"
-  float* red = reinterpret_cast<float*>(smem + L.red_off);  // [10][kConsumers]
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  float* red = reinterpret_cast<float*>(smem + L.red_off);  // [10][kThreads]
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   const long long units = geom.T * geom.n_g;
   const int box_bytes = geom.SC * geom.bw * IO::kBytes;
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kConsumerWarps);
+      mbar_init(empty0 + 8 * s, kWarps);
     }
-    mbar_init(redbar, kConsumerWarps);
-    mbar_init(redbar + 8, kConsumerWarps);
+    mbar_init(redbar, kWarps);
+    mbar_init(redbar + 8, kWarps);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
+    prefetch_map(&mx);
+    prefetch_map(&mdy);
   }
   __syncthreads();
 
-  if (warp == 0) {
-    if (lane != 0) return;
-    prefetch_map(&mx);
-    prefetch_map(&mdy);
-    prefetch_map(&mdx);
-    bool ok = true;
-    long long q = 0;
-    // coordinates of the chunk held by each stage (for its store)
-    int st_col[kBwdStages], st_row[kBwdStages];
-#pragma unroll
-    for (int s = 0; s < kBwdStages; ++s) st_col[s] = st_row[s] = 0;
-    for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
-      const long long tile = u / geom.n_g;
-      const int g = (int)(u - tile * geom.n_g);
-      const int nck = unit_chunks(geom, tile);
-      float cv[10];
+  // issue cursor (thread 0): unit iu, chunk ick of nick, sequence number iq
+  long long iu = blockIdx.x, iq = 0;
+  int ick = 0, inck = 0;
+  float cv[10];
+  auto start_unit = [&]() {
+    if (iu < units) {
+      const long long tile = iu / geom.n_g;
+      const int g = (int)(iu - tile * geom.n_g);
+      inck = unit_chunks(geom, tile);
 #pragma unroll
       for (int i = 0; i < 6; ++i) cv[i] = __ldg(a + g * 6 + i);
 #pragma unroll
       for (int j = 0; j < 4; ++j) cv[6 + j] = __ldg(b + g * 4 + j);
-      for (int ck = 0; ck < nck; ++ck, ++q) {
-        const int s = (int)(q % kBwdStages);
-        const uint32_t kq = (uint32_t)(q / kBwdStages);
-        unsigned char* stage = smem + s * L.stage_stride;
-        if (q >= kBwdStages) {
-          if (!mbar_wait(empty0 + 8 * s, (kq - 1) & 1)) { report(kErrEmptyWait); ok = false; break; }
-          for (int bx = 0; bx < geom.nbox; ++bx)
-            tma_store_2d(&mdx, st_col[s] + bx * geom.bw, st_row[s],
-                         smem_addr(stage + cbytes + bx * box_bytes));
-          bulk_commit();
-          bulk_wait_read_all();
-        }
-        float* cs = coef + s * kCoefSlot;
-#pragma unroll
-        for (int k = 0; k < 10; ++k) cs[k] = cv[k];
-        const int col = g * geom.dg;
-        const int row = (int)(tile * (long long)geom.SC * geom.chunks_per_unit + (long long)ck * geom.SC);
-        st_col[s] = col;
-        st_row[s] = row;
-        mbar_arrive_expect_tx(full0 + 8 * s, 2u * geom.chunk_bytes);
-        for (int bx = 0; bx < geom.nbox; ++bx) {
-          tma_load_2d(smem_addr(stage + bx * box_bytes), &mx, col + bx * geom.bw, row, full0 + 8 * s);
-          tma_load_2d(smem_addr(stage + cbytes + bx * box_bytes), &mdy, col + bx * geom.bw, row,
-                      full0 + 8 * s);
-        }
-      }
     }
-    if (ok) {
-      const long long first = q > kBwdStages ? q - kBwdStages : 0;
-      for (long long j = first; j < q; ++j) {
-        const int s = (int)(j % kBwdStages);
-        if (!mbar_wait(empty0 + 8 * s, (uint32_t)(j / kBwdStages) & 1)) {
+  };
+  auto issue = [&]() {
+    const int s = (int)(iq % kBwdStages);
+    const long long tile = iu / geom.n_g;
+    const int g = (int)(iu - tile * geom.n_g);
+    unsigned char* stage = smem + s * L.stage_stride;
+    float* cs = coef + s * kCoefSlot;
+#pragma unroll
+    for (int k = 0; k < 10; ++k) cs[k] = cv[k];
+    const int col = g * geom.dg;
+    const int row = (int)(tile * (long long)geom.SC * geom.chunks_per_unit + (long long)ick * geom.SC);
+    mbar_arrive_expect_tx(full0 + 8 * s, 2u * geom.chunk_bytes);
+    for (int bx = 0; bx < geom.nbox; ++bx) {
+      tma_load_2d(smem_addr(stage + bx * box_bytes), &mx, col + bx * geom.bw, row, full0 + 8 * s);
+      tma_load_2d(smem_addr(stage + cbytes + bx * box_bytes), &mdy, col + bx * geom.bw, row,
+                  full0 + 8 * s);
+    }
+    ++iq;
+    if (++ick == inck) {
+      ick = 0;
+      iu += gridDim.x;
+      start_unit();
+    }
+  };
+  if (tid == 0) {
+    start_unit();
+    for (int s = 0; s < kBwdStages && iu < units; ++s) issue();
+  }
+
+  VecMap<IO> vm;
+  vm.init(geom, tid);
+  const int nvec = (int)(geom.chunk_bytes / 16);
+  Coef54 c;
+  Acc54 acc;
+  bool ok = true;
+  long long q = 0;
+  uint32_t nred = 0;  // reductions done (phase of the reduction barriers)
+  for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const long long tile = u / geom.n_g;
+    const int g = (int)(u - tile * geom.n_g);
+    const int nck = unit_chunks(geom, tile);
+    const long long S = (long long)geom.SC * geom.chunks_per_unit;
+    acc.zero();
+    for (int ck = 0; ck < nck; ++ck, ++q) {
+      const int s = (int)(q % kBwdStages);
+      if (tid == 0 && q >= 1 && iu < units) {
+        if (!mbar_wait(empty0 + 8 * (int)((q - 1) % kBwdStages),
+                       (uint32_t)((q - 1) / kBwdStages) & 1)) {
           report(kErrEmptyWait);
           ok = false;
           break;
         }
-        unsigned char* stage = smem + s * L.stage_stride;
-        for (int bx = 0; bx < geom.nbox; ++bx)
-          tma_store_2d(&mdx, st_col[s] + bx * geom.bw, st_row[s],
-                       smem_addr(stage + cbytes + bx * box_bytes));
-        bulk_commit();
+        issue();
       }
-    }
-    if (!ok) {
-      const long long first = q > kBwdStages ? q - kBwdStages : 0;
-      for (long long j = first; j < q; ++j) {
-        if (!mbar_wait(full0 + 8 * (int)(j % kBwdStages), (uint32_t)(j / kBwdStages) & 1))
-          report(kErrDrainWait);
+      if (!mbar_wait(full0 + 8 * s, (uint32_t)(q / kBwdStages) & 1)) {
+        report(kErrFullWait);
+        ok = false;
+        break;
       }
-    }
-    bulk_wait_all();
-    return;
-  }
-
-  // consumers
-  const int ct = threadIdx.x - 32;
-  const int nvec = (int)(geom.chunk_bytes / 16);
-  Coef54 c;
-  Acc54 acc;
-  long long q = 0;
-  uint32_t nred = 0;  // reductions done (phase of the reduction barriers)
-  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-    const long long tile = u / geom.n_g;
-    const int g = (int)(u - tile * geom.n_g);
-    const int nck = unit_chunks(geom, tile);
-    acc.zero();
-    for (int ck = 0; ck < nck; ++ck, ++q) {
-      const int s = (int)(q % kBwdStages);
-      const uint32_t kq = (uint32_t)(q / kBwdStages);
-      if (!mbar_wait(full0 + 8 * s, kq & 1)) { report(kErrFullWait); return; }
       if (ck == 0) c.set(coef + s * kCoefSlot);
       const uint4* xb = reinterpret_cast<const uint4*>(smem + s * L.stage_stride);
-      uint4* gb = reinterpret_cast<uint4*>(smem + s * L.stage_stride + cbytes);
-      uint4 xv[kMaxVecPerThread], gv[kMaxVecPerThread];
+      const uint4* gb = reinterpret_cast<const uint4*>(smem + s * L.stage_stride + cbytes);
+      uint4 xv[kVec], gv[kVec];
 #pragma unroll
-      for (int it = 0; it < kMaxVecPerThread; ++it) {
-        const int vi = ct + it * kConsumers;
+      for (int it = 0; it < kVec; ++it) {
+        const int vi = tid + it * kThreads;
         if (vi < nvec) {
           xv[it] = xb[vi];
           gv[it] = gb[vi];
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
+      const long long row0 = tile * S + (long long)ck * geom.SC;
+      typename IO::T* dxo = dx + row0 * geom.d + (long long)g * geom.dg;
 #pragma unroll
-      for (int it = 0; it < kMaxVecPerThread; ++it) {
-        const int vi = ct + it * kConsumers;
-        if (vi < nvec) {
+      for (int it = 0; it < kVec; ++it) {
+        // rows past the end were zero-filled by TMA: they add exact zeros to
+        // the sums but must not be stored
+        if (tid + it * kThreads < nvec) {
           uint4 o;
           if constexpr (IO::kBytes == 2) {
             o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
@@ -584,54 +568,64 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
             o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
                            __float_as_uint(p1.y));
           }
-          gb[vi] = o;
+          if (row0 + vm.row[it] < geom.rows) store16(dxo + vm.off[it], o);
         }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
+    if (!ok) break;
 
     // Unit reduction, fixed order: lanes of a pair, then red[k][thread], then
-    // each warp sums coefficient k over threads lane, lane+32, ... (8 values in
-    // order) and an xor butterfly.
-    float* rk = red + ct;
-    rk[0 * kConsumers] = acc.a0.x + acc.a0.y;
-    rk[1 * kConsumers] = acc.a1.x + acc.a1.y;
-    rk[2 * kConsumers] = acc.a2.x + acc.a2.y;
-    rk[3 * kConsumers] = acc.a3.x + acc.a3.y;
-    rk[4 * kConsumers] = acc.a4.x + acc.a4.y;
-    rk[5 * kConsumers] = acc.a5.x + acc.a5.y;
-    rk[6 * kConsumers] = acc.b1.x + acc.b1.y;
-    rk[7 * kConsumers] = acc.b2.x + acc.b2.y;
-    rk[8 * kConsumers] = acc.b3.x + acc.b3.y;
-    rk[9 * kConsumers] = acc.b4.x + acc.b4.y;
+    // warp k sums coefficient k over threads lane, lane + 32, ... (in order)
+    // and an xor butterfly.
+    float* rk = red + tid;
+    rk[0 * kThreads] = acc.a0.x + acc.a0.y;
+    rk[1 * kThreads] = acc.a1.x + acc.a1.y;
+    rk[2 * kThreads] = acc.a2.x + acc.a2.y;
+    rk[3 * kThreads] = acc.a3.x + acc.a3.y;
+    rk[4 * kThreads] = acc.a4.x + acc.a4.y;
+    rk[5 * kThreads] = acc.a5.x + acc.a5.y;
+    rk[6 * kThreads] = acc.b1.x + acc.b1.y;
+    rk[7 * kThreads] = acc.b2.x + acc.b2.y;
+    rk[8 * kThreads] = acc.b3.x + acc.b3.y;
+    rk[9 * kThreads] = acc.b4.x + acc.b4.y;
     __syncwarp();
     if (lane == 0) mbar_arrive(redbar);
-    if (!mbar_wait(redbar, nred & 1)) { report(kErrReduceWait); return; }
-    const int cw = warp - 1;
-    for (int k = cw; k < 10; k += kConsumerWarps) {
-      const float* col = red + k * kConsumers;
+    if (!mbar_wait(redbar, nred & 1)) {
+      report(kErrReduceWait);
+      ok = false;
+      break;
+    }
+    for (int k = warp; k < 10; k += kWarps) {
+      const float* col = red + k * kThreads;
       float v = col[lane];
 #pragma unroll
-      for (int i = 1; i < kConsumerWarps; ++i) v += col[lane + 32 * i];
+      for (int i = 1; i < kWarps; ++i) v += col[lane + 32 * i];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) ws[((long long)g * 10 + k) * geom.T + tile] = v;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(redbar + 8);
-    if (!mbar_wait(redbar + 8, nred & 1)) { report(kErrReduceWait); return; }
+    if (!mbar_wait(redbar + 8, nred & 1)) {
+      report(kErrReduceWait);
+      ok = false;
+      break;
+    }
     ++nred;
+  }
+  if (!ok && tid == 0) {
+    for (long long j = q; j < iq; ++j)
+      if (!mbar_wait(full0 + 8 * (int)(j % kBwdStages), (uint32_t)(j / kBwdStages) & 1))
+        report(kErrDrainWait);
   }
 }
 
 // --- host-side launchers ---------------------------------------------------------
 
 // Raise a kernel's dynamic shared-memory limit to the largest layout it can
-// need. One cache per kernel instantiation (the instantiations share a
-// function-pointer type, so the cache is keyed on the template arguments);
-// set once per device.
+// need and ask for the largest shared-memory carveout. One cache per kernel
+// instantiation (the instantiations share a function-pointer type, so the
+// cache is keyed on the template arguments); set once per device.
 template <class IO, bool kBackward>
 inline cudaError_t ensure_smem(unsigned most) {
   static int done_for_device = -1;
@@ -639,50 +633,53 @@ inline cudaError_t ensure_smem(unsigned most) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (done_for_device == dev) return cudaSuccess;
-  if (kBackward)
-    e = cudaFuncSetAttribute(bwd_tma<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
-  else
-    e = cudaFuncSetAttribute(fwd_tma<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+  const void* fn = kBackward ? reinterpret_cast<const void*>(bwd_tma<IO>)
+                             : reinterpret_cast<const void*>(fwd_tma<IO>);
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done_for_device = dev;
   return e;
 }
 
-inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
-                                  const CUtensorMap& my, const float* a, const float* b, int sms,
-                                  cudaStream_t st) {
+inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx, void* y,
+                                  const float* a, const float* b, int sms, cudaStream_t st) {
   const Layout L(g.chunk_bytes, 1, kFwdStages, false);
   const unsigned most = Layout(kMaxChunkBytes, 1, kFwdStages, false).total;
   if (L.total > most) return cudaErrorInvalidValue;
   const long long items = ((g.rows + g.SC - 1) / g.SC) * g.n_g;
-  long long grid = (long long)kCtasPerSm * sms;
+  long long grid = sms;
   if (grid > items) grid = items;
   cudaError_t e;
   if (bf16) {
-    if ((e = (ensure_smem<IoBF16, false>(most))) != cudaSuccess) return e;
-    fwd_tma<IoBF16><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, my, a, b, g);
+    if ((e = ensure_smem<IoBF16, false>(most)) != cudaSuccess) return e;
+    fwd_tma<IoBF16><<<(unsigned)grid, kThreads, L.total, st>>>(mx, (IoBF16::T*)y, a, b, g);
   } else {
-    if ((e = (ensure_smem<IoF32, false>(most))) != cudaSuccess) return e;
-    fwd_tma<IoF32><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, my, a, b, g);
+    if ((e = ensure_smem<IoF32, false>(most)) != cudaSuccess) return e;
+    fwd_tma<IoF32><<<(unsigned)grid, kThreads, L.total, st>>>(mx, (IoF32::T*)y, a, b, g);
   }
   return cudaGetLastError();
 }
 
 inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
-                                  const CUtensorMap& mdy, const CUtensorMap& mdx, const float* a,
+                                  const CUtensorMap& mdy, void* dx, const float* a,
                                   const float* b, float* ws, int sms, cudaStream_t st) {
   const Layout L(g.chunk_bytes, 2, kBwdStages, true);
   const unsigned most = Layout(kMaxChunkBytes, 2, kBwdStages, true).total;
   if (L.total > most) return cudaErrorInvalidValue;
   const long long units = g.T * g.n_g;
-  long long grid = (long long)kCtasPerSm * sms;
+  long long grid = sms;
   if (grid > units) grid = units;
   cudaError_t e;
   if (bf16) {
-    if ((e = (ensure_smem<IoBF16, true>(most))) != cudaSuccess) return e;
-    bwd_tma<IoBF16><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, mdy, mdx, a, b, ws, g);
+    if ((e = ensure_smem<IoBF16, true>(most)) != cudaSuccess) return e;
+    bwd_tma<IoBF16><<<(unsigned)grid, kThreads, L.total, st>>>(mx, mdy, (IoBF16::T*)dx, a, b,
+                                                                ws, g);
   } else {
-    if ((e = (ensure_smem<IoF32, true>(most))) != cudaSuccess) return e;
-    bwd_tma<IoF32><<<(unsigned)grid, kTmaThreads, L.total, st>>>(mx, mdy, mdx, a, b, ws, g);
+    if ((e = ensure_smem<IoF32, true>(most)) != cudaSuccess) return e;
+    bwd_tma<IoF32><<<(unsigned)grid, kThreads, L.total, st>>>(mx, mdy, (IoF32::T*)dx, a, b, ws,
+                                                               g);
   }
   return cudaGetLastError();
 }
