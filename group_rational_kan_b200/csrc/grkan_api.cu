@@ -32,20 +32,49 @@ grkan_status_t cuda_status(cudaError_t e, const char* where) {
   return GRKAN_ERR_CUDA;
 }
 
-// Work partition. A "chunk" is SC rows of one group (about 12 KiB of one
-// tensor); a unit (row tile x group) is kChunksPerUnit chunks. The partition
-// depends only on the shape, never on the device, so the float32 partials --
-// and therefore dA and dB -- are the same bits on every run.
-constexpr long long kChunkBytes = GRK_CHUNK_BYTES;
-constexpr int kChunksPerUnit = 4;
+// Work partition. The backward reduces over (row tile x group) units of S rows;
+// S depends only on the shape, never on the device or the pointers, so the
+// float32 partials -- and therefore dA and dB -- are the same bits on every run.
+// For shapes the TMA kernels take, a unit is grk::kBoxesPerUnit TMA boxes of
+// the backward (SCw rows x bw channels, about 1.5 KiB); otherwise about 12 KiB
+// of rows of one group.
+constexpr long long kGenericTileBytes = 12288;
 constexpr int kMaxBoxRows = 256;
+
+struct Box {
+  int bw = 0;   // channels (0: no box fits)
+  int scw = 0;  // rows
+  int nbox = 0; // boxes per group row
+  unsigned bytes = 0;
+};
+
+// The largest box at most `target` bytes: width the largest divisor of d_g
+// that is at most 256 elements, a whole number of 16-byte vectors and fits,
+// height as many rows as fit (at most 256).
+Box choose_box(long long dg, int es, unsigned target) {
+  Box b;
+  if (dg <= 0) return b;
+  for (long long w = dg < 256 ? dg : 256; w >= 1; --w) {
+    if (dg % w == 0 && (w * es) % 16 == 0 && (unsigned)(w * es) <= target) {
+      b.bw = (int)w;
+      break;
+    }
+  }
+  if (b.bw == 0) return b;
+  long long rows = target / (unsigned)(b.bw * es);
+  if (rows > kMaxBoxRows) rows = kMaxBoxRows;
+  b.scw = (int)rows;
+  b.nbox = (int)(dg / b.bw);
+  b.bytes = (unsigned)(b.scw * b.bw * es);
+  return b;
+}
 
 struct Plan {
   long long rows = 0, d = 0, dg = 0;
   int n_g = 1, m = 0, n = 0, K = 1, es = 4;
   grkan_dtype_t dtype = GRKAN_F32;
-  int SC = 1;       // rows per chunk
-  int S = 1;        // rows per tile (unit)
+  Box fbox, bbox;   // forward / backward TMA boxes
+  long long S = 1;  // rows per tile (unit)
   long long T = 0;  // number of row tiles
   size_t ws_bytes = 0;
 };
@@ -69,12 +98,19 @@ grkan_status_t make_plan(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m
   p->K = m + 1 + n;
   p->dtype = dtype;
   p->es = dtype == GRKAN_F32 ? 4 : 2;
-  const long long row_bytes = p->dg * p->es;
-  long long sc = row_bytes > 0 ? kChunkBytes / row_bytes : kMaxBoxRows;
-  if (sc < 1) sc = 1;
-  if (sc > kMaxBoxRows) sc = kMaxBoxRows;
-  p->SC = (int)sc;
-  p->S = p->SC * kChunksPerUnit;
+  p->fbox = choose_box(p->dg, p->es, grk::kFwdBoxBytes);
+  p->bbox = choose_box(p->dg, p->es, grk::kBwdBoxBytes);
+  if (p->bbox.bw > 0) {
+    int per = grk::kBoxesPerUnit / p->bbox.nbox;
+    if (per < 1) per = 1;
+    p->S = (long long)p->bbox.scw * per;
+  } else {
+    const long long row_bytes = p->dg * p->es;
+    long long s = row_bytes > 0 ? kGenericTileBytes / row_bytes : kMaxBoxRows;
+    if (s < 1) s = 1;
+    if (s > kMaxBoxRows) s = kMaxBoxRows;
+    p->S = s;
+  }
   p->T = (rows + p->S - 1) / p->S;
   if (rows == 0 || d == 0) p->T = 0;
   p->ws_bytes = (size_t)p->T * (size_t)n_g * (size_t)p->K * sizeof(float);
@@ -114,7 +150,7 @@ cudaError_t launch_generic_fwd(const Plan& p, const void* x, void* y, const floa
   const long long units = p.T * p.n_g;
   grk::fwd_generic<IO, GRKAN_MAX_M, GRKAN_MAX_N><<<(unsigned)units, grk::kGenericThreads, 0, st>>>(
       (const typename IO::T*)x, (typename IO::T*)y, a, b, p.rows, p.d, (int)p.dg, p.n_g, p.m, p.n,
-      p.S);
+      (int)p.S);
   return cudaGetLastError();
 }
 
@@ -124,16 +160,15 @@ cudaError_t launch_generic_bwd(const Plan& p, const void* x, const void* dy, voi
   const long long units = p.T * p.n_g;
   grk::bwd_generic<IO, GRKAN_MAX_M, GRKAN_MAX_N><<<(unsigned)units, grk::kGenericThreads, 0, st>>>(
       (const typename IO::T*)x, (const typename IO::T*)dy, (typename IO::T*)dx, a, b, ws, p.rows,
-      p.d, (int)p.dg, p.n_g, p.m, p.n, p.S, p.T);
+      p.d, (int)p.dg, p.n_g, p.m, p.n, (int)p.S, p.T);
   return cudaGetLastError();
 }
 
 cudaError_t launch_merge(const Plan& p, const float* ws, float* dA, float* dB, double* sums64,
                          cudaStream_t st) {
   const long long outs = (long long)p.n_g * p.K;
-  const unsigned blocks = (unsigned)((outs + grk::kMergeWarps - 1) / grk::kMergeWarps);
-  grk::merge_partials<<<blocks, grk::kMergeWarps * 32, 0, st>>>(ws, dA, dB, sums64, p.T, p.n_g,
-                                                                 p.m, p.n);
+  grk::merge_partials<<<(unsigned)outs, grk::kMergeThreads, 0, st>>>(ws, dA, dB, sums64, p.T,
+                                                                      p.n_g, p.m, p.n);
   return cudaGetLastError();
 }
 
@@ -141,26 +176,13 @@ cudaError_t launch_merge(const Plan& p, const float* ws, float* dA, float* dB, d
 
 bool tma_degree_supported(int m, int n) { return grk::tma_has_degree(m, n); }
 
-// Box width for the TMA tensor maps: the largest divisor of d_g that is at most
-// 256 elements with a whole number of 16-byte units. 0 if none.
-int tma_box_width(const Plan& p) {
-  if (p.dg <= 0) return 0;
-  for (long long w = p.dg < 256 ? p.dg : 256; w >= 1; --w) {
-    if (p.dg % w == 0 && (w * p.es) % 16 == 0) return (int)w;
-  }
-  return 0;
-}
-
 bool tma_shape_ok(const Plan& p) {
   if (p.rows <= 0 || p.d <= 0) return false;
   if ((p.d * p.es) % 16 != 0 || (p.dg * p.es) % 16 != 0) return false;
   if (p.rows > 0x7fffffffLL || p.d > 0x7fffffffLL) return false;
-  const int bw = tma_box_width(p);
-  if (bw == 0) return false;
-  // a chunk (SC rows x d_g) fits one stage, and every TMA box inside it starts
-  // on a 128-byte boundary of shared memory
-  if ((long long)p.SC * p.dg * p.es > (long long)grk::kMaxChunkBytes) return false;
-  return ((long long)p.SC * bw * p.es) % 128 == 0;
+  // both boxes exist and every box starts on a 128-byte shared-memory boundary
+  // (slots are rounded up to 128 bytes)
+  return p.fbox.bw > 0 && p.bbox.bw > 0;
 }
 
 int choose_fwd_path(const Plan& p, const void* x, const void* y, uint32_t flags) {
@@ -199,8 +221,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over the (rows, d) tensor, box = (bw columns, SC rows).
-bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
+// 2-D map over the (rows, d) tensor, box = (bw columns, scw rows).
+bool make_map(CUtensorMap* map, const void* base, const Plan& p, const Box& bx) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_last_error("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled not found", 0);
@@ -208,7 +230,7 @@ bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
   }
   const cuuint64_t dims[2] = {(cuuint64_t)p.d, (cuuint64_t)p.rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(p.d * p.es)};
-  const cuuint32_t box[2] = {(cuuint32_t)bw, (cuuint32_t)p.SC};
+  const cuuint32_t box[2] = {(cuuint32_t)bx.bw, (cuuint32_t)bx.scw};
   const cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType dt =
       p.dtype == GRKAN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -219,18 +241,18 @@ bool make_map(CUtensorMap* map, const void* base, const Plan& p, int bw) {
   return r == CUDA_SUCCESS;
 }
 
-grk::TmaGeom make_geom(const Plan& p, int bw) {
+grk::TmaGeom make_geom(const Plan& p, const Box& bx) {
   grk::TmaGeom g;
   g.rows = p.rows;
+  g.T = p.T;
   g.d = p.d;
+  g.S = p.S;
   g.dg = (int)p.dg;
   g.n_g = p.n_g;
-  g.SC = p.SC;
-  g.chunks_per_unit = kChunksPerUnit;
-  g.T = p.T;
-  g.bw = bw;
-  g.nbox = (int)(p.dg / bw);
-  g.chunk_bytes = (unsigned)(p.SC * p.dg * p.es);
+  g.SCw = bx.scw;
+  g.bw = bx.bw;
+  g.nbox = bx.nbox;
+  g.box_bytes = bx.bytes;
   g.m = p.m;
   g.n = p.n;
   return g;
@@ -250,20 +272,18 @@ int sm_count() {
 
 grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float* a,
                               const float* b, cudaStream_t st) {
-  const int bw = tma_box_width(p);
   CUtensorMap mx;
-  if (!make_map(&mx, x, p, bw)) return GRKAN_ERR_CUDA;
-  const grk::TmaGeom geom = make_geom(p, bw);
+  if (!make_map(&mx, x, p, p.fbox)) return GRKAN_ERR_CUDA;
+  const grk::TmaGeom geom = make_geom(p, p.fbox);
   cudaError_t e = grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, y, a, b, sm_count(), st);
   return cuda_status(e, "forward (TMA) launch");
 }
 
 grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx,
                               const float* a, const float* b, float* ws, cudaStream_t st) {
-  const int bw = tma_box_width(p);
   CUtensorMap mx, mdy;
-  if (!make_map(&mx, x, p, bw) || !make_map(&mdy, dy, p, bw)) return GRKAN_ERR_CUDA;
-  const grk::TmaGeom geom = make_geom(p, bw);
+  if (!make_map(&mx, x, p, p.bbox) || !make_map(&mdy, dy, p, p.bbox)) return GRKAN_ERR_CUDA;
+  const grk::TmaGeom geom = make_geom(p, p.bbox);
   cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, dx, a, b, ws,
                                       sm_count(), st);
   return cuda_status(e, "backward (TMA) launch");

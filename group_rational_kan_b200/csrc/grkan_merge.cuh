@@ -2,8 +2,7 @@
 //
 // The first stage leaves one float32 partial per (row tile, group,
 // coefficient). This kernel adds the T partials of each (group, coefficient)
-// in double precision in a fixed order -- lane l takes tiles l, l+32, ...,
-// then a fixed xor butterfly -- and writes dA / dB. This is the "single
+// in double precision in a fixed order and writes dA / dB. This is the "single
 // controllable merge step" that replaces scattered atomic updates ("PolyKAN:
 // Efficient Fused GPU Operators for Polynomial Kolmogorov-Arnold Network
 // Variants", abstract, technique (iii)); the order never depends on timing,
@@ -14,28 +13,35 @@
 
 namespace grk {
 
-constexpr int kMergeWarps = 4;
+constexpr int kMergeThreads = 256;
 
-__global__ void __launch_bounds__(kMergeWarps * 32)
+// One CTA per (group, coefficient): thread t adds tiles t, t + 256, ... in
+// float64, then the CTA adds the 256 thread sums in a fixed tree (xor
+// butterfly inside each warp, warps in index order).
+__global__ void __launch_bounds__(kMergeThreads)
 merge_partials(const float* __restrict__ ws, float* __restrict__ dA, float* __restrict__ dB,
                double* __restrict__ sums64, long long T, int n_g, int m, int n) {
+  __shared__ double part[kMergeThreads / 32];
   const int K = m + 1 + n;
-  const int lane = threadIdx.x & 31;
-  const long long o = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
-  if (o >= (long long)n_g * K) return;
+  const long long o = blockIdx.x;
   const float* p = ws + o * T;
   double s = 0.0;
-  for (long long t = lane; t < T; t += 32) s += (double)p[t];
+  for (long long t = threadIdx.x; t < T; t += kMergeThreads) s += (double)p[t];
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) tot += part[w];
     const int g = (int)(o / K);
     const int k = (int)(o - (long long)g * K);
     if (k <= m)
-      dA[(long long)g * (m + 1) + k] = (float)s;
+      dA[(long long)g * (m + 1) + k] = (float)tot;
     else
-      dB[(long long)g * n + (k - m - 1)] = (float)s;
-    if (sums64) sums64[o] = s;
+      dB[(long long)g * n + (k - m - 1)] = (float)tot;
+    if (sums64) sums64[o] = tot;
   }
 }
 

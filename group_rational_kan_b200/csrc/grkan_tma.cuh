@@ -32,39 +32,42 @@ namespace grk {
 
 struct TmaGeom {
   long long rows;       // B * N
-  long long T;          // row tiles
+  long long T;          // row tiles (units per group)
   long long d;          // channels (row length)
+  long long S;          // rows per tile
   int dg;               // channels per group
   int n_g;              // groups
-  int SC;               // rows per chunk (TMA box height)
-  int chunks_per_unit;  // chunks per row tile
+  int SCw;              // rows per TMA box
   int bw;               // TMA box width (channels)
-  int nbox;             // boxes per chunk row = dg / bw
-  unsigned chunk_bytes; // SC * dg * element size (one tensor)
+  int nbox;             // boxes per group row = dg / bw
+  unsigned box_bytes;   // SCw * bw * element size
   int m, n;             // degrees
 };
 
 // Launch shape (compile-time; the defaults are the tuned configuration).
+// One CTA of kWarps independent warps per SM; every warp owns kFwdStages /
+// kBwdStages box slots of kFwdBoxBytes / kBwdBoxBytes per tensor.
 #ifndef GRK_WARPS
 #define GRK_WARPS 16
 #endif
 #ifndef GRK_FWD_STAGES
-#define GRK_FWD_STAGES 8
+#define GRK_FWD_STAGES 4
 #endif
 #ifndef GRK_BWD_STAGES
 #define GRK_BWD_STAGES 4
-#endif
-#ifndef GRK_CHUNK_BYTES
-#define GRK_CHUNK_BYTES 24576
 #endif
 
 constexpr int kWarps = GRK_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kFwdStages = GRK_FWD_STAGES;
 constexpr int kBwdStages = GRK_BWD_STAGES;
-constexpr unsigned kMaxChunkBytes = GRK_CHUNK_BYTES;
-constexpr int kVec = (int)((kMaxChunkBytes / 16 + kThreads - 1) / kThreads);  // vectors/thread
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;                 // 2 s
+constexpr unsigned kFwdBoxBytes = 32 * 6 * 16;  // 6 vectors of 16 bytes per lane
+constexpr unsigned kBwdBoxBytes = 32 * 3 * 16;  // 3 vectors per lane and tensor
+#ifndef GRK_BOXES_PER_UNIT
+#define GRK_BOXES_PER_UNIT 8
+#endif
+constexpr int kBoxesPerUnit = GRK_BOXES_PER_UNIT;  // backward boxes per (tile, group) unit
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 
 // Error codes written to g_grkan_device_error (bit-or).
 constexpr unsigned kErrFullWait = 1u;
@@ -232,62 +235,55 @@ __device__ __forceinline__ float2 bwd_pair(const Coef54& c, float2 x, float2 dy,
   return fma2(nu, dQ, mul2(t, dP));
 }
 
-// --- shared-memory layout ------------------------------------------------------
-
-constexpr int kCoefSlot = 16;  // floats per stage header (10 used)
-
 __host__ __device__ constexpr unsigned round_up(unsigned v, unsigned a) {
   return (v + a - 1) / a * a;
 }
 
-// [stages x tensors x chunk] [stages x header coef] [full bars] [empty bars]
-// [two reduction bars] [reduction buffer 10 x kThreads floats]
-struct Layout {
-  unsigned stage_stride;  // bytes of one stage (all tensors)
-  unsigned coef_off, bar_off, red_off, total;
-  __host__ __device__ Layout(unsigned chunk_bytes, int tensors, int stages, bool reduce) {
-    const unsigned cb = round_up(chunk_bytes, 128);
-    stage_stride = cb * (unsigned)tensors;
-    coef_off = stage_stride * (unsigned)stages;
-    bar_off = coef_off + (unsigned)(stages * kCoefSlot * 4);
-    red_off = round_up(bar_off + (unsigned)(2 * stages + 2) * 8, 128);
-    total = red_off + (reduce ? (unsigned)(10 * kThreads * 4) : 0u);
+// --- per-warp pipeline geometry ----------------------------------------------------
+//
+// Every warp runs its own pipeline: it owns kStages stage slots in shared
+// memory, each holding one TMA box (SCw rows x bw channels) of every input
+// tensor, and its own full / empty mbarriers. Nothing couples the warps of a
+// CTA after initialisation, so they drift out of phase and one warp's loads
+// and reductions overlap another's arithmetic.
+
+constexpr int kCoefFloats = 16;  // per-warp coefficient slot (10 used)
+
+// Per-warp shared memory: [stages][tensors][box, 128-byte rounded],
+// coefficient slot, then the 8-byte barriers.
+struct WarpLayout {
+  unsigned box_slot;   // bytes of one box slot
+  unsigned stage;      // bytes of one stage (all tensors)
+  unsigned coef_off;   // coefficient slot
+  unsigned bar_off;    // full[stages] then empty[stages]
+  unsigned per_warp;   // bytes per warp (multiple of 128)
+  __host__ __device__ WarpLayout(unsigned box_bytes, int tensors, int stages) {
+    box_slot = round_up(box_bytes, 128);
+    stage = box_slot * (unsigned)tensors;
+    coef_off = stage * (unsigned)stages;
+    bar_off = coef_off + kCoefFloats * 4;
+    per_warp = round_up(bar_off + (unsigned)(2 * stages) * 8, 128);
   }
 };
 
-// Chunks in unit (tile): ceil(min(S, rows - tile*S) / SC).
-__device__ __forceinline__ int unit_chunks(const TmaGeom& g, long long tile) {
-  const long long S = (long long)g.SC * g.chunks_per_unit;
-  long long left = g.rows - tile * S;
-  if (left > S) left = S;
-  return (int)((left + g.SC - 1) / g.SC);
-}
-
-// Where the vectors a thread owns in every chunk go in global memory. The
-// chunk is stored in shared memory as nbox boxes of SC rows x bw channels;
-// vector v (16 bytes) of the chunk is box v / (SC*vpr), row (v % (SC*vpr)) /
-// vpr, vector column v % vpr. off = element offset from the chunk's origin
-// (first row, first channel of the group); row = row within the chunk, or a
-// huge value for a slot past the end of the chunk.
-template <class IO>
-struct VecMap {
-  long long off[kVec];
-  int row[kVec];
-  __device__ __forceinline__ void init(const TmaGeom& g, int tid) {
+// Where the vectors a lane owns in every box go in global memory: vector v of
+// the box (16 bytes) is row v / vpr, vector column v % vpr; off = element
+// offset from the box origin, row = row in the box (huge for unused slots).
+template <class IO, int NV>
+struct LaneMap {
+  int off[NV];
+  int row[NV];
+  __device__ __forceinline__ void init(const TmaGeom& g, int lane, long long d) {
     constexpr int ve = 16 / IO::kBytes;  // elements per vector
     const int vpr = g.bw / ve;
-    const int vpb = vpr * g.SC;
-    const int nvec = (int)(g.chunk_bytes / 16);
+    const int nvec = (int)(g.box_bytes / 16);
 #pragma unroll
-    for (int it = 0; it < kVec; ++it) {
-      const int v = tid + it * kThreads;
+    for (int it = 0; it < NV; ++it) {
+      const int v = lane + it * 32;
       if (v < nvec) {
-        const int bx = v / vpb;
-        const int rem = v - bx * vpb;
-        const int r = rem / vpr;
-        const int c = rem - r * vpr;
+        const int r = v / vpr;
         row[it] = r;
-        off[it] = (long long)r * g.d + (long long)bx * g.bw + (long long)c * ve;
+        off[it] = (int)((long long)r * d) + (v - r * vpr) * ve;
       } else {
         row[it] = 0x3fffffff;
         off[it] = 0;
@@ -300,101 +296,135 @@ __device__ __forceinline__ void store16(void* p, uint4 v) {
   __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
-// --- forward -----------------------------------------------------------------------
-// Work items are (row chunk, group) pairs, item w -> chunk w / n_g, group w % n_g,
-// taken by CTA i as w = i, i + grid, ...
+// Stage a group's coefficients a_0..a_5, b_1..b_4 in the warp's shared slot
+// and read them back on every lane.
+__device__ __forceinline__ void stage_coefficients(float* slot, const float* a, const float* b,
+                                                   int g, int lane, Coef54& c) {
+  if (lane < 6) slot[lane] = __ldg(a + g * 6 + lane);
+  else if (lane < 10) slot[lane] = __ldg(b + g * 4 + (lane - 6));
+  __syncwarp();
+  c.set(slot);
+  __syncwarp();
+}
+
+// Sum ten per-lane values over the warp in a fixed order; every lane ends with
+// all ten sums. Recursive halving: at each step a lane keeps half of its
+// values (those of its own half of the index range) and adds the partner's.
+__device__ __forceinline__ void warp_sum10(float (&v)[16], int lane) {
+  // 16 slots, 10 used (the rest are zero)
+#pragma unroll
+  for (int step = 0; step < 4; ++step) {
+    const int half = 8 >> step;       // values kept after this step
+    const int mask = 16 >> step;      // partner distance
+    const bool upper = (lane & mask) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, mask);
+      v[i] = (upper ? v[i + half] : v[i]) + recv;
+    }
+  }
+  // now lane holds, in v[0], the sum over lanes l with l & 1 == lane & 1 ...
+  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+// --- forward -------------------------------------------------------------------------
+// Work items are boxes: item w -> (row block w / (n_g*nbox), group, box), taken
+// by warp gw of the grid as w = gw, gw + total warps, ...
+
+constexpr int kFwdVec = 6;  // vectors per lane in a forward box (3 KiB boxes)
 
 template <class IO>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  const Layout L(geom.chunk_bytes, 1, kFwdStages, false);
-  float* coef = reinterpret_cast<float*>(smem + L.coef_off);
-  const uint32_t full0 = smem_addr(smem + L.bar_off);
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const WarpLayout L(geom.box_bytes, 1, kFwdStages);
+  unsigned char* base = smem + warp * L.per_warp;
+  float* cslot = reinterpret_cast<float*>(base + L.coef_off);
+  const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * kFwdStages;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const long long row_chunks = (geom.rows + geom.SC - 1) / geom.SC;
-  const long long items = row_chunks * geom.n_g;
-  const int box_bytes = geom.SC * geom.bw * IO::kBytes;
+  const long long row_blocks = (geom.rows + geom.SCw - 1) / geom.SCw;
+  const long long per_rb = (long long)geom.n_g * geom.nbox;
+  const long long items = row_blocks * per_rb;
+  const long long gw = (long long)blockIdx.x * kWarps + warp;
+  const long long GW = (long long)gridDim.x * kWarps;
 
-  if (tid == 0) {
+  if (lane == 0) {
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kWarps);
+      mbar_init(empty0 + 8 * s, 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
-    prefetch_map(&mx);
+    if (warp == 0) prefetch_map(&mx);
   }
-  __syncthreads();
+  __syncwarp();
 
-  // issue cursor (thread 0): next item to load and its sequence number
-  long long iw = blockIdx.x, iq = 0;
+  long long iw = gw, iq = 0;  // issue cursor (lane 0)
   auto issue = [&]() {
     const int s = (int)(iq % kFwdStages);
-    const long long rc = iw / geom.n_g;
-    const int g = (int)(iw - rc * geom.n_g);
-    float* cs = coef + s * kCoefSlot;
-#pragma unroll
-    for (int i = 0; i < 6; ++i) cs[i] = __ldg(a + g * 6 + i);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) cs[6 + j] = __ldg(b + g * 4 + j);
-    mbar_arrive_expect_tx(full0 + 8 * s, geom.chunk_bytes);
-    for (int bx = 0; bx < geom.nbox; ++bx)
-      tma_load_2d(smem_addr(smem + s * L.stage_stride + bx * box_bytes), &mx,
-                  g * geom.dg + bx * geom.bw, (int)(rc * geom.SC), full0 + 8 * s);
-    iw += gridDim.x;
+    const long long rb = iw / per_rb;
+    const int rem = (int)(iw - rb * per_rb);
+    const int g = rem / geom.nbox;
+    const int bx = rem - g * geom.nbox;
+    mbar_arrive_expect_tx(full0 + 8 * s, geom.box_bytes);
+    tma_load_2d(smem_addr(base + s * L.stage), &mx, g * geom.dg + bx * geom.bw,
+                (int)(rb * geom.SCw), full0 + 8 * s);
+    iw += GW;
     ++iq;
   };
-  if (tid == 0)
+  if (lane == 0)
     for (int s = 0; s < kFwdStages && iw < items; ++s) issue();
+  __syncwarp();
 
-  VecMap<IO> vm;
-  vm.init(geom, tid);
-  const int nvec = (int)(geom.chunk_bytes / 16);
+  LaneMap<IO, kFwdVec> lm;
+  lm.init(geom, lane, geom.d);
   Coef54 c;
   int cur_g = -1;
   bool ok = true;
   long long q = 0;
-  for (long long w = blockIdx.x; w < items; w += gridDim.x, ++q) {
+  for (long long w = gw; w < items; w += GW, ++q) {
     const int s = (int)(q % kFwdStages);
-    if (tid == 0 && q >= 1 && iw < items) {
-      // refill the stage of chunk q-1 once every warp has read it
-      if (!mbar_wait(empty0 + 8 * (int)((q - 1) % kFwdStages),
-                     (uint32_t)((q - 1) / kFwdStages) & 1)) {
-        report(kErrEmptyWait);
-        ok = false;
-        break;
-      }
-      issue();
-    }
-    if (!mbar_wait(full0 + 8 * s, (uint32_t)(q / kFwdStages) & 1)) {
+    const uint32_t ph = (uint32_t)(q / kFwdStages) & 1;
+    if (!mbar_wait(full0 + 8 * s, ph)) {
       report(kErrFullWait);
       ok = false;
       break;
     }
-    const long long rc = w / geom.n_g;
-    const int g = (int)(w - rc * geom.n_g);
+    const long long rb = w / per_rb;
+    const int rem = (int)(w - rb * per_rb);
+    const int g = rem / geom.nbox;
+    const int bx = rem - g * geom.nbox;
     if (g != cur_g) {
-      c.set(coef + s * kCoefSlot);
+      stage_coefficients(cslot, a, b, g, lane, c);
       cur_g = g;
     }
-    const uint4* buf = reinterpret_cast<const uint4*>(smem + s * L.stage_stride);
-    uint4 v[kVec];
+    const uint4* buf = reinterpret_cast<const uint4*>(base + s * L.stage);
+    uint4 v[kFwdVec];
 #pragma unroll
-    for (int it = 0; it < kVec; ++it) {
-      const int vi = tid + it * kThreads;
-      if (vi < nvec) v[it] = buf[vi];
-    }
+    for (int it = 0; it < kFwdVec; ++it)
+      if (lm.row[it] < geom.SCw) v[it] = buf[lane + 32 * it];
+    // release the slot and refill it with the item kFwdStages ahead
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * s);
-    const long long row0 = rc * geom.SC;
-    typename IO::T* yo = y + row0 * geom.d + (long long)g * geom.dg;
+    if (lane == 0) {
+      mbar_arrive(empty0 + 8 * s);
+      if (iw < items) {
+        if (!mbar_wait(empty0 + 8 * s, ph)) {
+          report(kErrEmptyWait);
+          ok = false;
+        } else {
+          issue();
+        }
+      }
+    }
+    const long long row0 = rb * geom.SCw;
+    typename IO::T* yo = y + row0 * geom.d + (long long)g * geom.dg + (long long)bx * geom.bw;
 #pragma unroll
-    for (int it = 0; it < kVec; ++it) {
-      if (row0 + vm.row[it] < geom.rows) {
+    for (int it = 0; it < kFwdVec; ++it) {
+      if (row0 + lm.row[it] < geom.rows) {
         uint4 o;
         if constexpr (IO::kBytes == 2) {
           o.x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].x)));
@@ -409,11 +439,13 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
           o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
                          __float_as_uint(p1.y));
         }
-        store16(yo + vm.off[it], o);
+        store16(yo + lm.off[it], o);
       }
     }
+    ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+    if (!ok) break;
   }
-  if (!ok && tid == 0) {
+  if (!ok && lane == 0) {
     // wind down: let every issued load land before the CTA's memory goes away
     for (long long j = q; j < iq; ++j)
       if (!mbar_wait(full0 + 8 * (int)(j % kFwdStages), (uint32_t)(j / kFwdStages) & 1))
@@ -422,8 +454,18 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
 }
 
 // --- backward ------------------------------------------------------------------------
-// Units u = tile * n_g + g, taken by CTA i as u = i, i + grid, ...; the partial
-// sum of unit (tile, g), coefficient k goes to ws[(g * 10 + k) * T + tile].
+// Units u = tile * n_g + g (tile = S rows), taken by warp gw of the grid as
+// u = gw, gw + total warps, ...; a unit's boxes are its row blocks (SCw rows)
+// times the group's column boxes. The partial sum of unit (tile, g),
+// coefficient k goes to ws[(g * 10 + k) * T + tile].
+
+constexpr int kBwdVec = 3;  // vectors per lane in a backward box (1.5 KiB boxes)
+
+__device__ __forceinline__ int unit_boxes(const TmaGeom& g, long long tile) {
+  long long left = g.rows - tile * g.S;
+  if (left > g.S) left = g.S;
+  return (int)((left + g.SCw - 1) / g.SCw) * g.nbox;
+}
 
 template <class IO>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -431,189 +473,154 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         typename IO::T* __restrict__ dx, const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  const Layout L(geom.chunk_bytes, 2, kBwdStages, true);
-  const unsigned cbytes = round_up(geom.chunk_bytes, 128);  // x at +0, dy at +cbytes
-  float* coef = reinterpret_cast<float*>(smem + L.coef_off);
-  const uint32_t full0 = smem_addr(smem + L.bar_off);
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const WarpLayout L(geom.box_bytes, 2, kBwdStages);
+  unsigned char* base = smem + warp * L.per_warp;
+  float* cslot = reinterpret_cast<float*>(base + L.coef_off);
+  const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * kBwdStages;
-  const uint32_t redbar = empty0 + 8 * kBwdStages;  // two: "written", "read"
-  float* red = reinterpret_cast<float*>(smem + L.red_off);  // [10][kThreads]
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
   const long long units = geom.T * geom.n_g;
-  const int box_bytes = geom.SC * geom.bw * IO::kBytes;
+  const long long gw = (long long)blockIdx.x * kWarps + warp;
+  const long long GW = (long long)gridDim.x * kWarps;
 
-  if (tid == 0) {
+  if (lane == 0) {
     for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kWarps);
+      mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(redbar, kWarps);
-    mbar_init(redbar + 8, kWarps);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
-    prefetch_map(&mx);
-    prefetch_map(&mdy);
-  }
-  __syncthreads();
-
-  // issue cursor (thread 0): unit iu, chunk ick of nick, sequence number iq
-  long long iu = blockIdx.x, iq = 0;
-  int ick = 0, inck = 0;
-  float cv[10];
-  auto start_unit = [&]() {
-    if (iu < units) {
-      const long long tile = iu / geom.n_g;
-      const int g = (int)(iu - tile * geom.n_g);
-      inck = unit_chunks(geom, tile);
-#pragma unroll
-      for (int i = 0; i < 6; ++i) cv[i] = __ldg(a + g * 6 + i);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) cv[6 + j] = __ldg(b + g * 4 + j);
+    if (warp == 0) {
+      prefetch_map(&mx);
+      prefetch_map(&mdy);
     }
-  };
+  }
+  __syncwarp();
+
+  // issue cursor (lane 0): unit iu, box ib of inb, sequence number iq
+  long long iu = gw, iq = 0;
+  int ib = 0, inb = (gw < units) ? unit_boxes(geom, gw / geom.n_g) : 0;
   auto issue = [&]() {
     const int s = (int)(iq % kBwdStages);
     const long long tile = iu / geom.n_g;
     const int g = (int)(iu - tile * geom.n_g);
-    unsigned char* stage = smem + s * L.stage_stride;
-    float* cs = coef + s * kCoefSlot;
-#pragma unroll
-    for (int k = 0; k < 10; ++k) cs[k] = cv[k];
-    const int col = g * geom.dg;
-    const int row = (int)(tile * (long long)geom.SC * geom.chunks_per_unit + (long long)ick * geom.SC);
-    mbar_arrive_expect_tx(full0 + 8 * s, 2u * geom.chunk_bytes);
-    for (int bx = 0; bx < geom.nbox; ++bx) {
-      tma_load_2d(smem_addr(stage + bx * box_bytes), &mx, col + bx * geom.bw, row, full0 + 8 * s);
-      tma_load_2d(smem_addr(stage + cbytes + bx * box_bytes), &mdy, col + bx * geom.bw, row,
-                  full0 + 8 * s);
-    }
+    const int rb = ib / geom.nbox;
+    const int bx = ib - rb * geom.nbox;
+    const int col = g * geom.dg + bx * geom.bw;
+    const int row = (int)(tile * geom.S + (long long)rb * geom.SCw);
+    unsigned char* st = base + s * L.stage;
+    mbar_arrive_expect_tx(full0 + 8 * s, 2u * geom.box_bytes);
+    tma_load_2d(smem_addr(st), &mx, col, row, full0 + 8 * s);
+    tma_load_2d(smem_addr(st + L.box_slot), &mdy, col, row, full0 + 8 * s);
     ++iq;
-    if (++ick == inck) {
-      ick = 0;
-      iu += gridDim.x;
-      start_unit();
+    if (++ib == inb) {
+      ib = 0;
+      iu += GW;
+      inb = (iu < units) ? unit_boxes(geom, iu / geom.n_g) : 0;
     }
   };
-  if (tid == 0) {
-    start_unit();
+  if (lane == 0)
     for (int s = 0; s < kBwdStages && iu < units; ++s) issue();
-  }
+  __syncwarp();
 
-  VecMap<IO> vm;
-  vm.init(geom, tid);
-  const int nvec = (int)(geom.chunk_bytes / 16);
+  LaneMap<IO, kBwdVec> lm;
+  lm.init(geom, lane, geom.d);
   Coef54 c;
   Acc54 acc;
   bool ok = true;
   long long q = 0;
-  uint32_t nred = 0;  // reductions done (phase of the reduction barriers)
-  for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
+  for (long long u = gw; u < units && ok; u += GW) {
     const long long tile = u / geom.n_g;
     const int g = (int)(u - tile * geom.n_g);
-    const int nck = unit_chunks(geom, tile);
-    const long long S = (long long)geom.SC * geom.chunks_per_unit;
+    const int nb = unit_boxes(geom, tile);
+    stage_coefficients(cslot, a, b, g, lane, c);
     acc.zero();
-    for (int ck = 0; ck < nck; ++ck, ++q) {
+    for (int ibx = 0; ibx < nb; ++ibx, ++q) {
       const int s = (int)(q % kBwdStages);
-      if (tid == 0 && q >= 1 && iu < units) {
-        if (!mbar_wait(empty0 + 8 * (int)((q - 1) % kBwdStages),
-                       (uint32_t)((q - 1) / kBwdStages) & 1)) {
-          report(kErrEmptyWait);
-          ok = false;
-          break;
-        }
-        issue();
-      }
-      if (!mbar_wait(full0 + 8 * s, (uint32_t)(q / kBwdStages) & 1)) {
+      const uint32_t ph = (uint32_t)(q / kBwdStages) & 1;
+      if (!mbar_wait(full0 + 8 * s, ph)) {
         report(kErrFullWait);
         ok = false;
         break;
       }
-      if (ck == 0) c.set(coef + s * kCoefSlot);
-      const uint4* xb = reinterpret_cast<const uint4*>(smem + s * L.stage_stride);
-      const uint4* gb = reinterpret_cast<const uint4*>(smem + s * L.stage_stride + cbytes);
-      uint4 xv[kVec], gv[kVec];
+      const uint4* xb = reinterpret_cast<const uint4*>(base + s * L.stage);
+      const uint4* gb = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot);
+      uint4 xv[kBwdVec], gv[kBwdVec];
 #pragma unroll
-      for (int it = 0; it < kVec; ++it) {
-        const int vi = tid + it * kThreads;
-        if (vi < nvec) {
-          xv[it] = xb[vi];
-          gv[it] = gb[vi];
+      for (int it = 0; it < kBwdVec; ++it) {
+        if (lm.row[it] < geom.SCw) {
+          xv[it] = xb[lane + 32 * it];
+          gv[it] = gb[lane + 32 * it];
+        } else {
+          xv[it] = make_uint4(0, 0, 0, 0);
+          gv[it] = make_uint4(0, 0, 0, 0);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * s);
-      const long long row0 = tile * S + (long long)ck * geom.SC;
-      typename IO::T* dxo = dx + row0 * geom.d + (long long)g * geom.dg;
-#pragma unroll
-      for (int it = 0; it < kVec; ++it) {
-        // rows past the end were zero-filled by TMA: they add exact zeros to
-        // the sums but must not be stored
-        if (tid + it * kThreads < nvec) {
-          uint4 o;
-          if constexpr (IO::kBytes == 2) {
-            o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
-            o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
-            o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
-            o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
+      if (lane == 0) {
+        mbar_arrive(empty0 + 8 * s);
+        if (iu < units) {
+          if (!mbar_wait(empty0 + 8 * s, ph)) {
+            report(kErrEmptyWait);
+            ok = false;
           } else {
-            const float2 p0 = bwd_pair(
-                c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
-                make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
-            const float2 p1 = bwd_pair(
-                c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
-                make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
-            o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
-                           __float_as_uint(p1.y));
+            issue();
           }
-          if (row0 + vm.row[it] < geom.rows) store16(dxo + vm.off[it], o);
         }
       }
+      const int rb = ibx / geom.nbox;
+      const int bx = ibx - rb * geom.nbox;
+      const long long row0 = tile * geom.S + (long long)rb * geom.SCw;
+      typename IO::T* dxo =
+          dx + row0 * geom.d + (long long)g * geom.dg + (long long)bx * geom.bw;
+#pragma unroll
+      for (int it = 0; it < kBwdVec; ++it) {
+        // rows past the end arrive zero-filled from TMA: they add exact zeros
+        // to the sums and are not stored
+        uint4 o;
+        if constexpr (IO::kBytes == 2) {
+          o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
+          o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
+          o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
+          o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
+        } else {
+          const float2 p0 = bwd_pair(
+              c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
+              make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
+          const float2 p1 = bwd_pair(
+              c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
+              make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
+          o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
+                         __float_as_uint(p1.y));
+        }
+        if (row0 + lm.row[it] < geom.rows) store16(dxo + lm.off[it], o);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+      if (!ok) break;
     }
     if (!ok) break;
-
-    // Unit reduction, fixed order: lanes of a pair, then red[k][thread], then
-    // warp k sums coefficient k over threads lane, lane + 32, ... (in order)
-    // and an xor butterfly.
-    float* rk = red + tid;
-    rk[0 * kThreads] = acc.a0.x + acc.a0.y;
-    rk[1 * kThreads] = acc.a1.x + acc.a1.y;
-    rk[2 * kThreads] = acc.a2.x + acc.a2.y;
-    rk[3 * kThreads] = acc.a3.x + acc.a3.y;
-    rk[4 * kThreads] = acc.a4.x + acc.a4.y;
-    rk[5 * kThreads] = acc.a5.x + acc.a5.y;
-    rk[6 * kThreads] = acc.b1.x + acc.b1.y;
-    rk[7 * kThreads] = acc.b2.x + acc.b2.y;
-    rk[8 * kThreads] = acc.b3.x + acc.b3.y;
-    rk[9 * kThreads] = acc.b4.x + acc.b4.y;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(redbar);
-    if (!mbar_wait(redbar, nred & 1)) {
-      report(kErrReduceWait);
-      ok = false;
-      break;
-    }
-    for (int k = warp; k < 10; k += kWarps) {
-      const float* col = red + k * kThreads;
-      float v = col[lane];
+    // Unit reduction, fixed order: the two lanes of each pair, then a
+    // recursive-halving exchange over the warp.
+    float v[16];
+    v[0] = acc.a0.x + acc.a0.y;
+    v[1] = acc.a1.x + acc.a1.y;
+    v[2] = acc.a2.x + acc.a2.y;
+    v[3] = acc.a3.x + acc.a3.y;
+    v[4] = acc.a4.x + acc.a4.y;
+    v[5] = acc.a5.x + acc.a5.y;
+    v[6] = acc.b1.x + acc.b1.y;
+    v[7] = acc.b2.x + acc.b2.y;
+    v[8] = acc.b3.x + acc.b3.y;
+    v[9] = acc.b4.x + acc.b4.y;
 #pragma unroll
-      for (int i = 1; i < kWarps; ++i) v += col[lane + 32 * i];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) ws[((long long)g * 10 + k) * geom.T + tile] = v;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(redbar + 8);
-    if (!mbar_wait(redbar + 8, nred & 1)) {
-      report(kErrReduceWait);
-      ok = false;
-      break;
-    }
-    ++nred;
+    for (int k = 10; k < 16; ++k) v[k] = 0.f;
+    warp_sum10(v, lane);
+    // after the exchange lane l holds the sum of coefficient (l >> 1) & 15
+    const int k = (lane >> 1) & 15;
+    if ((lane & 1) == 0 && k < 10) ws[((long long)g * 10 + k) * geom.T + tile] = v[0];
   }
-  if (!ok && tid == 0) {
+  if (!ok && lane == 0) {
     for (long long j = q; j < iq; ++j)
       if (!mbar_wait(full0 + 8 * (int)(j % kBwdStages), (uint32_t)(j / kBwdStages) & 1))
         report(kErrDrainWait);
@@ -622,12 +629,12 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 
 // --- host-side launchers ---------------------------------------------------------
 
-// Raise a kernel's dynamic shared-memory limit to the largest layout it can
-// need and ask for the largest shared-memory carveout. One cache per kernel
-// instantiation (the instantiations share a function-pointer type, so the
-// cache is keyed on the template arguments); set once per device.
+// Raise a kernel's dynamic shared-memory limit to what it uses and ask for the
+// largest shared-memory carveout. One cache per kernel instantiation (the
+// instantiations share a function-pointer type, so the cache is keyed on the
+// template arguments); set once per device.
 template <class IO, bool kBackward>
-inline cudaError_t ensure_smem(unsigned most) {
+inline cudaError_t ensure_smem(unsigned bytes) {
   static int done_for_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -635,7 +642,7 @@ inline cudaError_t ensure_smem(unsigned most) {
   if (done_for_device == dev) return cudaSuccess;
   const void* fn = kBackward ? reinterpret_cast<const void*>(bwd_tma<IO>)
                              : reinterpret_cast<const void*>(fwd_tma<IO>);
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared);
@@ -643,21 +650,24 @@ inline cudaError_t ensure_smem(unsigned most) {
   return e;
 }
 
+// Shared memory of a launch: kWarps per-warp regions of the largest box.
+inline unsigned fwd_smem_bytes() { return kWarps * WarpLayout(kFwdBoxBytes, 1, kFwdStages).per_warp; }
+inline unsigned bwd_smem_bytes() { return kWarps * WarpLayout(kBwdBoxBytes, 2, kBwdStages).per_warp; }
+
 inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx, void* y,
                                   const float* a, const float* b, int sms, cudaStream_t st) {
-  const Layout L(g.chunk_bytes, 1, kFwdStages, false);
-  const unsigned most = Layout(kMaxChunkBytes, 1, kFwdStages, false).total;
-  if (L.total > most) return cudaErrorInvalidValue;
-  const long long items = ((g.rows + g.SC - 1) / g.SC) * g.n_g;
+  if (g.box_bytes > kFwdBoxBytes) return cudaErrorInvalidValue;
+  const unsigned smem = fwd_smem_bytes();
+  const long long items = ((g.rows + g.SCw - 1) / g.SCw) * g.n_g * g.nbox;
   long long grid = sms;
-  if (grid > items) grid = items;
+  if (grid * kWarps > items) grid = (items + kWarps - 1) / kWarps;
   cudaError_t e;
   if (bf16) {
-    if ((e = ensure_smem<IoBF16, false>(most)) != cudaSuccess) return e;
-    fwd_tma<IoBF16><<<(unsigned)grid, kThreads, L.total, st>>>(mx, (IoBF16::T*)y, a, b, g);
+    if ((e = ensure_smem<IoBF16, false>(smem)) != cudaSuccess) return e;
+    fwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoBF16::T*)y, a, b, g);
   } else {
-    if ((e = ensure_smem<IoF32, false>(most)) != cudaSuccess) return e;
-    fwd_tma<IoF32><<<(unsigned)grid, kThreads, L.total, st>>>(mx, (IoF32::T*)y, a, b, g);
+    if ((e = ensure_smem<IoF32, false>(smem)) != cudaSuccess) return e;
+    fwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoF32::T*)y, a, b, g);
   }
   return cudaGetLastError();
 }
@@ -665,20 +675,19 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
 inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
                                   const CUtensorMap& mdy, void* dx, const float* a,
                                   const float* b, float* ws, int sms, cudaStream_t st) {
-  const Layout L(g.chunk_bytes, 2, kBwdStages, true);
-  const unsigned most = Layout(kMaxChunkBytes, 2, kBwdStages, true).total;
-  if (L.total > most) return cudaErrorInvalidValue;
+  if (g.box_bytes > kBwdBoxBytes) return cudaErrorInvalidValue;
+  const unsigned smem = bwd_smem_bytes();
   const long long units = g.T * g.n_g;
   long long grid = sms;
-  if (grid > units) grid = units;
+  if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
   cudaError_t e;
   if (bf16) {
-    if ((e = ensure_smem<IoBF16, true>(most)) != cudaSuccess) return e;
-    bwd_tma<IoBF16><<<(unsigned)grid, kThreads, L.total, st>>>(mx, mdy, (IoBF16::T*)dx, a, b,
+    if ((e = ensure_smem<IoBF16, true>(smem)) != cudaSuccess) return e;
+    bwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, mdy, (IoBF16::T*)dx, a, b,
                                                                 ws, g);
   } else {
-    if ((e = ensure_smem<IoF32, true>(most)) != cudaSuccess) return e;
-    bwd_tma<IoF32><<<(unsigned)grid, kThreads, L.total, st>>>(mx, mdy, (IoF32::T*)dx, a, b, ws,
+    if ((e = ensure_smem<IoF32, true>(smem)) != cudaSuccess) return e;
+    bwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, mdy, (IoF32::T*)dx, a, b, ws,
                                                                g);
   }
   return cudaGetLastError();
