@@ -328,9 +328,40 @@ __device__ __forceinline__ void warp_sum10(float (&v)[16], int lane) {
   v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
+// Mixed-radix counter (hi, mid, lo) with radices (unbounded, nmid, nlo), stepped
+// by a fixed stride without any division in the loop.
+struct Cursor3 {
+  long long hi;
+  int mid, lo;
+  long long s_hi;
+  int s_mid, s_lo, nmid, nlo;
+  __device__ __forceinline__ void init(long long first, long long stride, int nmid_, int nlo_) {
+    nmid = nmid_;
+    nlo = nlo_;
+    const long long per = (long long)nmid * nlo;
+    hi = first / per;
+    const int r = (int)(first - hi * per);
+    mid = r / nlo;
+    lo = r - mid * nlo;
+    s_hi = stride / per;
+    const int sr = (int)(stride - s_hi * per);
+    s_mid = sr / nlo;
+    s_lo = sr - s_mid * nlo;
+  }
+  __device__ __forceinline__ void next() {
+    lo += s_lo;
+    int carry = lo >= nlo;
+    lo -= carry ? nlo : 0;
+    mid += s_mid + carry;
+    carry = mid >= nmid;
+    mid -= carry ? nmid : 0;
+    hi += s_hi + carry;
+  }
+};
+
 // --- forward -------------------------------------------------------------------------
-// Work items are boxes: item w -> (row block w / (n_g*nbox), group, box), taken
-// by warp gw of the grid as w = gw, gw + total warps, ...
+// Work items are boxes (row block, group, column box), taken by warp gw of the
+// grid as item gw, gw + total warps, ... in row-block-major order.
 
 constexpr int kFwdVec = 6;  // vectors per lane in a forward box (3 KiB boxes)
 
@@ -347,8 +378,6 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * kFwdStages;
   const long long row_blocks = (geom.rows + geom.SCw - 1) / geom.SCw;
-  const long long per_rb = (long long)geom.n_g * geom.nbox;
-  const long long items = row_blocks * per_rb;
   const long long gw = (long long)blockIdx.x * kWarps + warp;
   const long long GW = (long long)gridDim.x * kWarps;
 
@@ -363,21 +392,19 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   }
   __syncwarp();
 
-  long long iw = gw, iq = 0;  // issue cursor (lane 0)
+  Cursor3 ic;  // issue cursor (lane 0): (row block, group, box)
+  ic.init(gw, GW, geom.n_g, geom.nbox);
+  int iq = 0;
   auto issue = [&]() {
-    const int s = (int)(iq % kFwdStages);
-    const long long rb = iw / per_rb;
-    const int rem = (int)(iw - rb * per_rb);
-    const int g = rem / geom.nbox;
-    const int bx = rem - g * geom.nbox;
+    const int s = iq % kFwdStages;
     mbar_arrive_expect_tx(full0 + 8 * s, geom.box_bytes);
-    tma_load_2d(smem_addr(base + s * L.stage), &mx, g * geom.dg + bx * geom.bw,
-                (int)(rb * geom.SCw), full0 + 8 * s);
-    iw += GW;
+    tma_load_2d(smem_addr(base + s * L.stage), &mx, ic.mid * geom.dg + ic.lo * geom.bw,
+                (int)(ic.hi * geom.SCw), full0 + 8 * s);
+    ic.next();
     ++iq;
   };
   if (lane == 0)
-    for (int s = 0; s < kFwdStages && iw < items; ++s) issue();
+    for (int s = 0; s < kFwdStages && ic.hi < row_blocks; ++s) issue();
   __syncwarp();
 
   LaneMap<IO, kFwdVec> lm;
@@ -385,19 +412,18 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   Coef54 c;
   int cur_g = -1;
   bool ok = true;
-  long long q = 0;
-  for (long long w = gw; w < items; w += GW, ++q) {
-    const int s = (int)(q % kFwdStages);
+  int q = 0;
+  Cursor3 cc;  // consumer cursor
+  cc.init(gw, GW, geom.n_g, geom.nbox);
+  for (; cc.hi < row_blocks; cc.next(), ++q) {
+    const int s = q % kFwdStages;
     const uint32_t ph = (uint32_t)(q / kFwdStages) & 1;
     if (!mbar_wait(full0 + 8 * s, ph)) {
       report(kErrFullWait);
       ok = false;
       break;
     }
-    const long long rb = w / per_rb;
-    const int rem = (int)(w - rb * per_rb);
-    const int g = rem / geom.nbox;
-    const int bx = rem - g * geom.nbox;
+    const int g = cc.mid;
     if (g != cur_g) {
       stage_coefficients(cslot, a, b, g, lane, c);
       cur_g = g;
@@ -411,7 +437,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(empty0 + 8 * s);
-      if (iw < items) {
+      if (ic.hi < row_blocks) {
         if (!mbar_wait(empty0 + 8 * s, ph)) {
           report(kErrEmptyWait);
           ok = false;
@@ -420,8 +446,8 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
         }
       }
     }
-    const long long row0 = rb * geom.SCw;
-    typename IO::T* yo = y + row0 * geom.d + (long long)g * geom.dg + (long long)bx * geom.bw;
+    const long long row0 = cc.hi * geom.SCw;
+    typename IO::T* yo = y + row0 * geom.d + (g * geom.dg + cc.lo * geom.bw);
 #pragma unroll
     for (int it = 0; it < kFwdVec; ++it) {
       if (row0 + lm.row[it] < geom.rows) {
@@ -447,24 +473,25 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   }
   if (!ok && lane == 0) {
     // wind down: let every issued load land before the CTA's memory goes away
-    for (long long j = q; j < iq; ++j)
-      if (!mbar_wait(full0 + 8 * (int)(j % kFwdStages), (uint32_t)(j / kFwdStages) & 1))
+    for (int j = q; j < iq; ++j)
+      if (!mbar_wait(full0 + 8 * (j % kFwdStages), (uint32_t)(j / kFwdStages) & 1))
         report(kErrDrainWait);
   }
 }
 
 // --- backward ------------------------------------------------------------------------
-// Units u = tile * n_g + g (tile = S rows), taken by warp gw of the grid as
-// u = gw, gw + total warps, ...; a unit's boxes are its row blocks (SCw rows)
-// times the group's column boxes. The partial sum of unit (tile, g),
-// coefficient k goes to ws[(g * 10 + k) * T + tile].
+// Units (tile, g) (tile = S rows) are taken by warp gw of the grid as unit
+// gw, gw + total warps, ... in tile-major order; a unit's boxes are its row
+// blocks (SCw rows) times the group's column boxes. The partial sum of unit
+// (tile, g), coefficient k goes to ws[(g * 10 + k) * T + tile].
 
 constexpr int kBwdVec = 3;  // vectors per lane in a backward box (1.5 KiB boxes)
 
-__device__ __forceinline__ int unit_boxes(const TmaGeom& g, long long tile) {
+// Row blocks of tile `tile`: ceil(min(S, rows - tile * S) / SCw).
+__device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile) {
   long long left = g.rows - tile * g.S;
   if (left > g.S) left = g.S;
-  return (int)((left + g.SCw - 1) / g.SCw) * g.nbox;
+  return (int)((left + g.SCw - 1) / g.SCw);
 }
 
 template <class IO>
@@ -480,7 +507,6 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   float* cslot = reinterpret_cast<float*>(base + L.coef_off);
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * kBwdStages;
-  const long long units = geom.T * geom.n_g;
   const long long gw = (long long)blockIdx.x * kWarps + warp;
   const long long GW = (long long)gridDim.x * kWarps;
 
@@ -498,30 +524,31 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   }
   __syncwarp();
 
-  // issue cursor (lane 0): unit iu, box ib of inb, sequence number iq
-  long long iu = gw, iq = 0;
-  int ib = 0, inb = (gw < units) ? unit_boxes(geom, gw / geom.n_g) : 0;
+  // issue cursor (lane 0): unit (tile, g) = iu.hi, iu.lo; box (irb, ibx) of inrb row blocks
+  Cursor3 iu;
+  iu.init(gw, GW, 1, geom.n_g);
+  int irb = 0, ibx = 0, inrb = (iu.hi < geom.T) ? tile_row_blocks(geom, iu.hi) : 0;
+  int iq = 0;
   auto issue = [&]() {
-    const int s = (int)(iq % kBwdStages);
-    const long long tile = iu / geom.n_g;
-    const int g = (int)(iu - tile * geom.n_g);
-    const int rb = ib / geom.nbox;
-    const int bx = ib - rb * geom.nbox;
-    const int col = g * geom.dg + bx * geom.bw;
-    const int row = (int)(tile * geom.S + (long long)rb * geom.SCw);
+    const int s = iq % kBwdStages;
+    const int col = iu.lo * geom.dg + ibx * geom.bw;
+    const int row = (int)(iu.hi * geom.S) + irb * geom.SCw;
     unsigned char* st = base + s * L.stage;
     mbar_arrive_expect_tx(full0 + 8 * s, 2u * geom.box_bytes);
     tma_load_2d(smem_addr(st), &mx, col, row, full0 + 8 * s);
     tma_load_2d(smem_addr(st + L.box_slot), &mdy, col, row, full0 + 8 * s);
     ++iq;
-    if (++ib == inb) {
-      ib = 0;
-      iu += GW;
-      inb = (iu < units) ? unit_boxes(geom, iu / geom.n_g) : 0;
+    if (++ibx == geom.nbox) {
+      ibx = 0;
+      if (++irb == inrb) {
+        irb = 0;
+        iu.next();
+        inrb = (iu.hi < geom.T) ? tile_row_blocks(geom, iu.hi) : 0;
+      }
     }
   };
   if (lane == 0)
-    for (int s = 0; s < kBwdStages && iu < units; ++s) issue();
+    for (int s = 0; s < kBwdStages && iu.hi < geom.T; ++s) issue();
   __syncwarp();
 
   LaneMap<IO, kBwdVec> lm;
@@ -529,75 +556,78 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   Coef54 c;
   Acc54 acc;
   bool ok = true;
-  long long q = 0;
-  for (long long u = gw; u < units && ok; u += GW) {
-    const long long tile = u / geom.n_g;
-    const int g = (int)(u - tile * geom.n_g);
-    const int nb = unit_boxes(geom, tile);
+  int q = 0;
+  Cursor3 cu;
+  cu.init(gw, GW, 1, geom.n_g);
+  for (; cu.hi < geom.T && ok; cu.next()) {
+    const long long tile = cu.hi;
+    const int g = cu.lo;
+    const int nrb = tile_row_blocks(geom, tile);
     stage_coefficients(cslot, a, b, g, lane, c);
     acc.zero();
-    for (int ibx = 0; ibx < nb; ++ibx, ++q) {
-      const int s = (int)(q % kBwdStages);
-      const uint32_t ph = (uint32_t)(q / kBwdStages) & 1;
-      if (!mbar_wait(full0 + 8 * s, ph)) {
-        report(kErrFullWait);
-        ok = false;
-        break;
-      }
-      const uint4* xb = reinterpret_cast<const uint4*>(base + s * L.stage);
-      const uint4* gb = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot);
-      uint4 xv[kBwdVec], gv[kBwdVec];
-#pragma unroll
-      for (int it = 0; it < kBwdVec; ++it) {
-        if (lm.row[it] < geom.SCw) {
-          xv[it] = xb[lane + 32 * it];
-          gv[it] = gb[lane + 32 * it];
-        } else {
-          xv[it] = make_uint4(0, 0, 0, 0);
-          gv[it] = make_uint4(0, 0, 0, 0);
+    typename IO::T* dxt = dx + tile * geom.S * geom.d + g * geom.dg;
+    const long long rows_left = geom.rows - tile * geom.S;
+    for (int rb = 0; rb < nrb && ok; ++rb) {
+      for (int bx = 0; bx < geom.nbox; ++bx, ++q) {
+        const int s = q % kBwdStages;
+        const uint32_t ph = (uint32_t)(q / kBwdStages) & 1;
+        if (!mbar_wait(full0 + 8 * s, ph)) {
+          report(kErrFullWait);
+          ok = false;
+          break;
         }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(empty0 + 8 * s);
-        if (iu < units) {
-          if (!mbar_wait(empty0 + 8 * s, ph)) {
-            report(kErrEmptyWait);
-            ok = false;
+        const uint4* xb = reinterpret_cast<const uint4*>(base + s * L.stage);
+        const uint4* gb = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot);
+        uint4 xv[kBwdVec], gv[kBwdVec];
+#pragma unroll
+        for (int it = 0; it < kBwdVec; ++it) {
+          if (lm.row[it] < geom.SCw) {
+            xv[it] = xb[lane + 32 * it];
+            gv[it] = gb[lane + 32 * it];
           } else {
-            issue();
+            xv[it] = make_uint4(0, 0, 0, 0);
+            gv[it] = make_uint4(0, 0, 0, 0);
           }
         }
-      }
-      const int rb = ibx / geom.nbox;
-      const int bx = ibx - rb * geom.nbox;
-      const long long row0 = tile * geom.S + (long long)rb * geom.SCw;
-      typename IO::T* dxo =
-          dx + row0 * geom.d + (long long)g * geom.dg + (long long)bx * geom.bw;
-#pragma unroll
-      for (int it = 0; it < kBwdVec; ++it) {
-        // rows past the end arrive zero-filled from TMA: they add exact zeros
-        // to the sums and are not stored
-        uint4 o;
-        if constexpr (IO::kBytes == 2) {
-          o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
-          o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
-          o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
-          o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
-        } else {
-          const float2 p0 = bwd_pair(
-              c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
-              make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
-          const float2 p1 = bwd_pair(
-              c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
-              make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
-          o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
-                         __float_as_uint(p1.y));
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty0 + 8 * s);
+          if (iu.hi < geom.T) {
+            if (!mbar_wait(empty0 + 8 * s, ph)) {
+              report(kErrEmptyWait);
+              ok = false;
+            } else {
+              issue();
+            }
+          }
         }
-        if (row0 + lm.row[it] < geom.rows) store16(dxo + lm.off[it], o);
+        const int r0 = rb * geom.SCw;  // row of the box within the tile
+        typename IO::T* dxo = dxt + (long long)r0 * geom.d + bx * geom.bw;
+#pragma unroll
+        for (int it = 0; it < kBwdVec; ++it) {
+          // rows past the end arrive zero-filled from TMA: they add exact
+          // zeros to the sums and are not stored
+          uint4 o;
+          if constexpr (IO::kBytes == 2) {
+            o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
+            o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
+            o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
+            o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
+          } else {
+            const float2 p0 = bwd_pair(
+                c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
+                make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
+            const float2 p1 = bwd_pair(
+                c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
+                make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
+            o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
+                           __float_as_uint(p1.y));
+          }
+          if (r0 + lm.row[it] < rows_left) store16(dxo + lm.off[it], o);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        if (!ok) break;
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-      if (!ok) break;
     }
     if (!ok) break;
     // Unit reduction, fixed order: the two lanes of each pair, then a
@@ -621,8 +651,8 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     if ((lane & 1) == 0 && k < 10) ws[((long long)g * 10 + k) * geom.T + tile] = v[0];
   }
   if (!ok && lane == 0) {
-    for (long long j = q; j < iq; ++j)
-      if (!mbar_wait(full0 + 8 * (int)(j % kBwdStages), (uint32_t)(j / kBwdStages) & 1))
+    for (int j = q; j < iq; ++j)
+      if (!mbar_wait(full0 + 8 * (j % kBwdStages), (uint32_t)(j / kBwdStages) & 1))
         report(kErrDrainWait);
   }
 }
