@@ -56,6 +56,27 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
 
 
+def measured_traffic(w):
+    """DRAM bytes per backward launch from the committed ncu summary, scaled by
+    elements; None unless the summary covers this workload and the kernel
+    sources are the ones it was captured on."""
+    import hashlib
+    if w.name != "kat_b":
+        return None
+    try:
+        text = open(os.path.join(ROOT, "profiles", "bwd_tma_kat_b.md")).read()
+        per = float(text.split("traffic_bytes_per_element:")[1].split()[0])
+        want = text.split("kernel_source_sha256_16:")[1].split()[0]
+        h = hashlib.sha256()
+        for f in ("grkan_tma.cuh", "grkan_common.cuh"):
+            h.update(open(os.path.join(ROOT, "group_rational_kan_b200", "csrc", f), "rb").read())
+        if h.hexdigest()[:16] != want:
+            return None
+        return per * w.elems
+    except Exception:
+        return None
+
+
 def dtype_name(w):
     return "f32" if w.dtype == synth.F32 else "bf16"
 
@@ -189,6 +210,7 @@ def main():
     import torch
     import torch.distributed as dist
     import group_rational_kan_b200 as grk
+    from group_rational_kan_b200.dist import all_gather_sums
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -224,7 +246,6 @@ def main():
     ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
     K = m + 1 + n
     sums64 = torch.empty((n_g, K), dtype=torch.float64, device=dev) if world > 1 else None
-    gathered = torch.empty((world, n_g, K), dtype=torch.float64, device=dev) if world > 1 else None
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     path_f = grk.grkan_forward_path(x, y, B, N, d, n_g, m, n, dt)
@@ -247,8 +268,8 @@ def main():
         check(grk.grkan_backward_merge(ws, wsb, dA, dB, sums64, B, N, d, n_g, m, n, dt, sp),
               "backward_merge")
         if world > 1:
-            dist.all_gather_into_tensor(gathered, sums64)
-            check(grk.grkan_merge_ranks(gathered, world, dA, dB, n_g, m, n, sp), "merge_ranks")
+            g = all_gather_sums(sums64)
+            check(grk.grkan_merge_ranks(g, world, dA, dB, n_g, m, n, sp), "merge_ranks")
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -333,7 +354,10 @@ def main():
                                     "backward": "tma" if path_b == 1 else "generic"}),
         "roofline": {"bound": "hbm", "kernel": "backward stage 1 (dx + dA/dB partials)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                     "frac": achieved / peak, "traffic": measured_traffic(w),
+                     "traffic_note": "ncu dram read+write of a 25,000-row capture scaled by "
+                                     "elements (profiles/bwd_tma_kat_b.md)",
+                     "peak_source": peak_src,
                      "bytes_per_launch": bwd_bytes, "launch_ms": bwd_ms},
         "kernels": {
             "forward": {"ms": fwd_ms, "GB/s": fwd_bytes / (fwd_ms * 1e-3) / 1e9,

@@ -1,0 +1,52 @@
+"""Data-parallel exchange of the coefficient gradients over torch.distributed.
+
+Rows shard across ranks with no halo; the only exchange is dA / dB. Each rank
+merges its own partials to float64 sums (grkan_backward_merge with sums64), the
+ranks all-gather those n_g x (m+1+n) doubles, and every rank adds the gathered
+blocks in rank order (grkan_merge_ranks). The order never depends on the
+transport or the topology, so every rank holds bit-identical gradients, and the
+result is bit-reproducible from run to run.
+"""
+import torch
+import torch.distributed as dist
+
+
+def all_gather_sums(sums64: torch.Tensor, group=None) -> torch.Tensor:
+    """(n_g, K) float64 per rank -> (world, n_g, K), block r from rank r."""
+    world = dist.get_world_size(group)
+    flat = sums64.contiguous().view(-1)
+    out = torch.empty((world * flat.numel(),), dtype=sums64.dtype, device=sums64.device)
+    dist.all_gather_into_tensor(out, flat, group=group)
+    return out.view((world,) + tuple(sums64.shape))
+
+
+def data_parallel_backward(x, dy, a, b, n_g, group=None, dx=None, workspace=None, stream=None):
+    """Backward of this rank's rows, with dA / dB summed over every rank.
+
+    Returns (dx, dA, dB); dA and dB are identical bits on every rank."""
+    import group_rational_kan_b200 as grk
+    B, N, d, dt = grk._dims(x, n_g)
+    m = a.shape[-1] - 1
+    n = b.shape[-1] if b is not None else 0
+    K = m + 1 + n
+    if dx is None:
+        dx = torch.empty_like(x)
+    dA = torch.empty((n_g, m + 1), dtype=torch.float32, device=x.device)
+    dB = torch.empty((n_g, n), dtype=torch.float32, device=x.device)
+    wsb = grk.grkan_backward_workspace_bytes(B, N, d, n_g, m, n, dt)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=x.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    sums = torch.empty((n_g, K), dtype=torch.float64, device=x.device)
+    st = grk.grkan_backward_partials(x, dy, a, b, dx, B, N, d, n_g, m, n, dt, workspace, nbytes,
+                                     0, stream)
+    if st == 0:
+        st = grk.grkan_backward_merge(workspace, nbytes, dA, dB, sums, B, N, d, n_g, m, n, dt,
+                                      stream)
+    if st != 0:
+        raise grk.GrkanError(st, "data_parallel_backward")
+    gathered = all_gather_sums(sums, group)
+    st = grk.grkan_merge_ranks(gathered, gathered.shape[0], dA, dB, n_g, m, n, stream)
+    if st != 0:
+        raise grk.GrkanError(st, "grkan_merge_ranks")
+    return dx, dA, dB
