@@ -16,13 +16,14 @@ __all__ = [
     "GrkanError", "F32", "BF16", "FLAG_GENERIC", "lib", "library_path",
     "grkan_forward", "grkan_forward_ex", "grkan_backward", "grkan_backward_ex",
     "grkan_backward_partials", "grkan_backward_merge", "grkan_backward_workspace_bytes",
-    "grkan_merge_ranks",
+    "grkan_merge_ranks", "grkan_backward_noalloc", "NOALLOC_WORKSPACE_BYTES",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
     "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
 ]
 
 F32, BF16 = 0, 1
 FLAG_GENERIC = 1
+NOALLOC_WORKSPACE_BYTES = 4 << 20  # GRKAN_NOALLOC_WORKSPACE_BYTES
 ABI_VERSION = 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -63,6 +64,8 @@ def _load():
         "grkan_backward_merge": (S, [P, SZ, P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int,
                                      P]),
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
+        "grkan_backward_noalloc": (S, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
+                                       ctypes.c_int, P]),
         "grkan_forward_path": (I32, [P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int, U32]),
         "grkan_backward_path": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int, U32]),
         "grkan_device_error": (S, [P, P]),
@@ -154,6 +157,13 @@ def grkan_backward_merge(workspace, workspace_bytes, dA, dB, sums64, B, N, d, n_
 def grkan_merge_ranks(gathered, world, dA, dB, n_g, m, n, stream=None):
     return lib().grkan_merge_ranks(_ptr(gathered), world, _ptr(dA), _ptr(dB), n_g, m, n,
                                    _stream(stream))
+
+
+def grkan_backward_noalloc(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, stream=None):
+    """grkan_backward with the library's static scratch array as workspace (for
+    callers that cannot allocate device memory per call)."""
+    return lib().grkan_backward_noalloc(_ptr(x), _ptr(dy), _ptr(a), _ptr(b), _ptr(dx), _ptr(dA),
+                                        _ptr(dB), B, N, d, n_g, m, n, dtype, _stream(stream))
 
 
 def grkan_forward_path(x, y, B, N, d, n_g, m, n, dtype, flags=0):

@@ -346,6 +346,33 @@ grkan_status_t do_merge(const Plan& p, const void* ws, size_t ws_bytes, float* d
   return cuda_status(e, "merge launch");
 }
 
+// Scratch for grkan_backward_noalloc: file-scope static device memory, one copy
+// per device that loads the library. Host code must not pass the symbol itself
+// to a kernel (in host code it names a host-side stand-in); it looks up the
+// device address once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_ws[GRKAN_NOALLOC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_ws on the current device (looked up on first use).
+grkan_status_t noalloc_workspace(void** out) {
+  int dev = 0;
+  grkan_status_t s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != GRKAN_OK) return s;
+  if (dev < 0 || dev >= kMaxDevices) return GRKAN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    s = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_ws), "cudaGetSymbolAddress");
+    if (s != GRKAN_OK) return s;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GRKAN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -430,6 +457,31 @@ grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* d
   grk::merge_ranks<<<(unsigned)((per + threads - 1) / threads), threads, 0,
                      (cudaStream_t)stream>>>(gathered, world, dA, dB, n_g, m, n);
   return cuda_status(cudaGetLastError(), "merge_ranks launch");
+}
+
+grkan_status_t grkan_backward_noalloc(const void* x, const void* dy, const float* a,
+                                      const float* b, void* dx, float* dA, float* dB, int64_t B,
+                                      int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                                      grkan_dtype_t dtype, void* stream) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (!dA || (p.n > 0 && !dB)) return GRKAN_ERR_NULL;
+  if (p.ws_bytes > (size_t)GRKAN_NOALLOC_WORKSPACE_BYTES) {
+    set_last_error("grkan_backward_noalloc", "workspace needed exceeds the static scratch",
+                   (int)(p.ws_bytes >> 20));
+    return GRKAN_ERR_WORKSPACE;
+  }
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  void* ws = nullptr;
+  s = noalloc_workspace(&ws);
+  if (s != GRKAN_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.T > 0) {
+    s = do_partials(p, x, dy, a, b, dx, ws, GRKAN_NOALLOC_WORKSPACE_BYTES, 0u, st);
+    if (s != GRKAN_OK) return s;
+  }
+  return do_merge(p, ws, GRKAN_NOALLOC_WORKSPACE_BYTES, dA, dB, nullptr, st);
 }
 
 int32_t grkan_forward_path(const void* x, const void* y, int64_t B, int64_t N, int64_t d,

@@ -144,6 +144,28 @@ GRKAN_API grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world
                                            float* dB, int32_t n_g, int32_t m, int32_t n,
                                            void* stream);
 
+/* Backward without a caller-supplied workspace (no counterpart in the paper;
+ * an addition for callers that cannot allocate device memory per call, such as
+ * a plugin whose host framework owns all device memory and forbids allocation
+ * while enqueueing work, or a process that must keep its device footprint fixed
+ * after start-up). Same arguments and results as grkan_backward, minus the
+ * workspace: the partial sums go to a scratch array of
+ * GRKAN_NOALLOC_WORKSPACE_BYTES that the library holds in static device memory
+ * on every GPU that loads it, until the process exits. Shapes whose workspace
+ * (grkan_backward_workspace_bytes) exceeds that size return GRKAN_ERR_WORKSPACE.
+ * Nothing is allocated: the first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current, so make that first
+ * call before any stream capture. All calls share the one array: calls whose
+ * kernels overlap on the GPU (different streams without ordering) race and give
+ * wrong gradients; calls ordered on one stream are safe. The array keeps the
+ * last call's partials; every call overwrites all it reads. */
+#define GRKAN_NOALLOC_WORKSPACE_BYTES (4u << 20)
+GRKAN_API grkan_status_t grkan_backward_noalloc(const void* x, const void* dy, const float* a,
+                                                const float* b, void* dx, float* dA, float* dB,
+                                                int64_t B, int64_t N, int64_t d, int32_t n_g,
+                                                int32_t m, int32_t n, grkan_dtype_t dtype,
+                                                void* stream);
+
 /* Which kernels a call with these arguments would run: 1 = TMA-pipelined
  * persistent kernels, 0 = generic grid-stride kernels, < 0 = invalid arguments
  * (the negated status). x, y are only inspected for alignment. */
