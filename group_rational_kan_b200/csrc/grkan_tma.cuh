@@ -61,8 +61,16 @@ constexpr int kWarps = GRK_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kFwdStages = GRK_FWD_STAGES;
 constexpr int kBwdStages = GRK_BWD_STAGES;
-constexpr unsigned kFwdBoxBytes = 32 * 6 * 16;  // 6 vectors of 16 bytes per lane
-constexpr unsigned kBwdBoxBytes = 32 * 3 * 16;  // 3 vectors per lane and tensor
+#ifndef GRK_FWD_VEC
+#define GRK_FWD_VEC 6
+#endif
+#ifndef GRK_BWD_VEC
+#define GRK_BWD_VEC 3
+#endif
+constexpr int kFwdVec = GRK_FWD_VEC;  // 16-byte vectors per lane in a forward box
+constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor in a backward box
+constexpr unsigned kFwdBoxBytes = 32 * kFwdVec * 16;
+constexpr unsigned kBwdBoxBytes = 32 * kBwdVec * 16;
 #ifndef GRK_BOXES_PER_UNIT
 #define GRK_BOXES_PER_UNIT 8
 #endif
@@ -202,22 +210,13 @@ __device__ __forceinline__ float2 bwd_pair(const Coef54& c, float2 x, float2 dy,
   const float2 x3 = mul2(x2, x);
   const float2 x4 = mul2(x2, x2);
   const float2 x5 = mul2(x4, x);
-  float2 P = fma2(c.a1, x, c.a0);
-  P = fma2(c.a2, x2, P);
-  P = fma2(c.a3, x3, P);
-  P = fma2(c.a4, x4, P);
-  P = fma2(c.a5, x5, P);
-  float2 dP = fma2(c.ia2, x, c.a1);
-  dP = fma2(c.ia3, x2, dP);
-  dP = fma2(c.ia4, x3, dP);
-  dP = fma2(c.ia5, x4, dP);
-  float2 Q = mul2(c.b1, x);
-  Q = fma2(c.b2, x2, Q);
-  Q = fma2(c.b3, x3, Q);
-  Q = fma2(c.b4, x4, Q);
-  float2 dQ = fma2(c.jb2, x, c.b1);
-  dQ = fma2(c.jb3, x2, dQ);
-  dQ = fma2(c.jb4, x3, dQ);
+  // Estrin's scheme: P = (a0 + a1 x) + x^2 (a2 + a3 x) + x^4 (a4 + a5 x), and the
+  // same pairing for P', Q, Q' -- the operation count of the power form with
+  // dependency chains of three.
+  const float2 P = fma2(x4, fma2(c.a5, x, c.a4), fma2(x2, fma2(c.a3, x, c.a2), fma2(c.a1, x, c.a0)));
+  const float2 dP = fma2(x4, c.ia5, fma2(x2, fma2(c.ia4, x, c.ia3), fma2(c.ia2, x, c.a1)));
+  const float2 Q = fma2(x3, fma2(c.b4, x, c.b3), mul2(x, fma2(c.b2, x, c.b1)));
+  const float2 dQ = fma2(x2, fma2(c.jb4, x, c.jb3), fma2(c.jb2, x, c.b1));
   const float2 r = make_float2(rcp_approx(1.f + fabsf(Q.x)), rcp_approx(1.f + fabsf(Q.y)));
   const float2 y = mul2(P, r);
   const float2 t = mul2(dy, r);
@@ -363,7 +362,6 @@ struct Cursor3 {
 // Work items are boxes (row block, group, column box), taken by warp gw of the
 // grid as item gw, gw + total warps, ... in row-block-major order.
 
-constexpr int kFwdVec = 6;  // vectors per lane in a forward box (3 KiB boxes)
 
 template <class IO>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -485,7 +483,6 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
 // blocks (SCw rows) times the group's column boxes. The partial sum of unit
 // (tile, g), coefficient k goes to ws[(g * 10 + k) * T + tile].
 
-constexpr int kBwdVec = 3;  // vectors per lane in a backward box (1.5 KiB boxes)
 
 // Row blocks of tile `tile`: ceil(min(S, rows - tile * S) / SCw).
 __device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile) {
@@ -554,6 +551,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   LaneMap<IO, kBwdVec> lm;
   lm.init(geom, lane, geom.d);
   Coef54 c;
+  int cur_g = -1;
   Acc54 acc;
   bool ok = true;
   int q = 0;
@@ -563,7 +561,10 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     const long long tile = cu.hi;
     const int g = cu.lo;
     const int nrb = tile_row_blocks(geom, tile);
-    stage_coefficients(cslot, a, b, g, lane, c);
+    if (g != cur_g) {
+      stage_coefficients(cslot, a, b, g, lane, c);
+      cur_g = g;
+    }
     acc.zero();
     typename IO::T* dxt = dx + tile * geom.S * geom.d + g * geom.dg;
     const long long rows_left = geom.rows - tile * geom.S;
