@@ -67,10 +67,14 @@ constexpr int kBwdStages = GRK_BWD_STAGES;
 #ifndef GRK_BWD_VEC
 #define GRK_BWD_VEC 3
 #endif
+#ifndef GRK_BWD_HALVES
+#define GRK_BWD_HALVES 1
+#endif
 constexpr int kFwdVec = GRK_FWD_VEC;  // 16-byte vectors per lane in a forward box
-constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor in a backward box
+constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor, per pass
+constexpr int kBwdHalves = GRK_BWD_HALVES;  // passes over a backward box
 constexpr unsigned kFwdBoxBytes = 32 * kFwdVec * 16;
-constexpr unsigned kBwdBoxBytes = 32 * kBwdVec * 16;
+constexpr unsigned kBwdBoxBytes = 32 * kBwdVec * kBwdHalves * 16;
 #ifndef GRK_BOXES_PER_UNIT
 #define GRK_BOXES_PER_UNIT 8
 #endif
@@ -159,8 +163,11 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
+// Two bf16 -> float32 exactly: the low half moved to the top by a byte permute,
+// the high half by a mask (both integer-pipe operations).
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return make_float2(__uint_as_float(__byte_perm(w, 0u, 0x1044)),
+                     __uint_as_float(w & 0xffff0000u));
 }
 __device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) {
   __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);  // .x -> low half
@@ -548,7 +555,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     for (int s = 0; s < kBwdStages && iu.hi < geom.T; ++s) issue();
   __syncwarp();
 
-  LaneMap<IO, kBwdVec> lm;
+  LaneMap<IO, kBwdVec * kBwdHalves> lm;
   lm.init(geom, lane, geom.d);
   Coef54 c;
   int cur_g = -1;
@@ -579,52 +586,60 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         }
         const uint4* xb = reinterpret_cast<const uint4*>(base + s * L.stage);
         const uint4* gb = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot);
-        uint4 xv[kBwdVec], gv[kBwdVec];
-#pragma unroll
-        for (int it = 0; it < kBwdVec; ++it) {
-          if (lm.row[it] < geom.SCw) {
-            xv[it] = xb[lane + 32 * it];
-            gv[it] = gb[lane + 32 * it];
-          } else {
-            xv[it] = make_uint4(0, 0, 0, 0);
-            gv[it] = make_uint4(0, 0, 0, 0);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(empty0 + 8 * s);
-          if (iu.hi < geom.T) {
-            if (!mbar_wait(empty0 + 8 * s, ph)) {
-              report(kErrEmptyWait);
-              ok = false;
-            } else {
-              issue();
-            }
-          }
-        }
         const int r0 = rb * geom.SCw;  // row of the box within the tile
         typename IO::T* dxo = dxt + (long long)r0 * geom.d + bx * geom.bw;
 #pragma unroll
-        for (int it = 0; it < kBwdVec; ++it) {
-          // rows past the end arrive zero-filled from TMA: they add exact
-          // zeros to the sums and are not stored
-          uint4 o;
-          if constexpr (IO::kBytes == 2) {
-            o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
-            o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
-            o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
-            o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
-          } else {
-            const float2 p0 = bwd_pair(
-                c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
-                make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
-            const float2 p1 = bwd_pair(
-                c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
-                make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
-            o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
-                           __float_as_uint(p1.y));
+        for (int h = 0; h < kBwdHalves; ++h) {
+          uint4 xv[kBwdVec], gv[kBwdVec];
+#pragma unroll
+          for (int it = 0; it < kBwdVec; ++it) {
+            const int sl = h * kBwdVec + it;
+            if (lm.row[sl] < geom.SCw) {
+              xv[it] = xb[lane + 32 * sl];
+              gv[it] = gb[lane + 32 * sl];
+            } else {
+              xv[it] = make_uint4(0, 0, 0, 0);
+              gv[it] = make_uint4(0, 0, 0, 0);
+            }
           }
-          if (r0 + lm.row[it] < rows_left) store16(dxo + lm.off[it], o);
+          if (h == kBwdHalves - 1) {
+            // release the slot (every lane has read it) and refill it
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(empty0 + 8 * s);
+              if (iu.hi < geom.T) {
+                if (!mbar_wait(empty0 + 8 * s, ph)) {
+                  report(kErrEmptyWait);
+                  ok = false;
+                } else {
+                  issue();
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int it = 0; it < kBwdVec; ++it) {
+            const int sl = h * kBwdVec + it;
+            // rows past the end arrive zero-filled from TMA: they add exact
+            // zeros to the sums and are not stored
+            uint4 o;
+            if constexpr (IO::kBytes == 2) {
+              o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
+              o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
+              o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
+              o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
+            } else {
+              const float2 p0 = bwd_pair(
+                  c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
+                  make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
+              const float2 p1 = bwd_pair(
+                  c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
+                  make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
+              o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
+                             __float_as_uint(p1.y));
+            }
+            if (r0 + lm.row[sl] < rows_left) store16(dxo + lm.off[sl], o);
+          }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
         if (!ok) break;
