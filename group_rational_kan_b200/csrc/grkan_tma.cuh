@@ -51,10 +51,10 @@ struct TmaGeom {
 #define GRK_WARPS 16
 #endif
 #ifndef GRK_FWD_STAGES
-#define GRK_FWD_STAGES 4
+#define GRK_FWD_STAGES 6
 #endif
 #ifndef GRK_BWD_STAGES
-#define GRK_BWD_STAGES 4
+#define GRK_BWD_STAGES 2
 #endif
 
 constexpr int kWarps = GRK_WARPS;
@@ -62,13 +62,13 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kFwdStages = GRK_FWD_STAGES;
 constexpr int kBwdStages = GRK_BWD_STAGES;
 #ifndef GRK_FWD_VEC
-#define GRK_FWD_VEC 6
+#define GRK_FWD_VEC 4
 #endif
 #ifndef GRK_BWD_VEC
 #define GRK_BWD_VEC 3
 #endif
 #ifndef GRK_BWD_HALVES
-#define GRK_BWD_HALVES 1
+#define GRK_BWD_HALVES 2
 #endif
 constexpr int kFwdVec = GRK_FWD_VEC;  // 16-byte vectors per lane in a forward box
 constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor, per pass
