@@ -98,8 +98,8 @@ grkan_status_t make_plan(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m
   p->K = m + 1 + n;
   p->dtype = dtype;
   p->es = dtype == GRKAN_F32 ? 4 : 2;
-  p->fbox = choose_box(p->dg, p->es, grk::kFwdBoxBytes);
-  p->bbox = choose_box(p->dg, p->es, grk::kBwdBoxBytes);
+  p->fbox = choose_box(p->dg, p->es, grk::fwd_box_target(dtype == GRKAN_BF16));
+  p->bbox = choose_box(p->dg, p->es, grk::bwd_box_target(dtype == GRKAN_BF16));
   if (p->bbox.bw > 0) {
     int per = grk::kBoxesPerUnit / p->bbox.nbox;
     if (per < 1) per = 1;

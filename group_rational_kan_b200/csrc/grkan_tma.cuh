@@ -45,36 +45,73 @@ struct TmaGeom {
 };
 
 // Launch shape (compile-time; the defaults are the tuned configuration).
-// One CTA of kWarps independent warps per SM; every warp owns kFwdStages /
-// kBwdStages box slots of kFwdBoxBytes / kBwdBoxBytes per tensor.
+// One CTA of kWarps independent warps per SM. Every warp owns, per element
+// type, a ring of forward stages (one box of x each) and of backward stages
+// (one box of x and one of dy each). float32 rows are HBM-bound: smaller boxes,
+// deeper rings. The bf16 backward is bound by the FMA pipe: 3 KiB boxes read in
+// two passes of three 16-byte vectors per lane, two stages.
 #ifndef GRK_WARPS
 #define GRK_WARPS 16
 #endif
-#ifndef GRK_FWD_STAGES
-#define GRK_FWD_STAGES 6
+#ifndef GRK_F32_FWD_VEC
+#define GRK_F32_FWD_VEC 6
 #endif
-#ifndef GRK_BWD_STAGES
-#define GRK_BWD_STAGES 2
+#ifndef GRK_F32_FWD_STAGES
+#define GRK_F32_FWD_STAGES 4
+#endif
+#ifndef GRK_F32_BWD_HALVES
+#define GRK_F32_BWD_HALVES 1
+#endif
+#ifndef GRK_F32_BWD_STAGES
+#define GRK_F32_BWD_STAGES 4
+#endif
+#ifndef GRK_BF16_FWD_VEC
+#define GRK_BF16_FWD_VEC 4
+#endif
+#ifndef GRK_BF16_FWD_STAGES
+#define GRK_BF16_FWD_STAGES 6
+#endif
+#ifndef GRK_BF16_BWD_HALVES
+#define GRK_BF16_BWD_HALVES 2
+#endif
+#ifndef GRK_BF16_BWD_STAGES
+#define GRK_BF16_BWD_STAGES 2
 #endif
 
 constexpr int kWarps = GRK_WARPS;
 constexpr int kThreads = kWarps * 32;
-constexpr int kFwdStages = GRK_FWD_STAGES;
-constexpr int kBwdStages = GRK_BWD_STAGES;
-#ifndef GRK_FWD_VEC
-#define GRK_FWD_VEC 4
-#endif
-#ifndef GRK_BWD_VEC
-#define GRK_BWD_VEC 3
-#endif
-#ifndef GRK_BWD_HALVES
-#define GRK_BWD_HALVES 2
-#endif
-constexpr int kFwdVec = GRK_FWD_VEC;  // 16-byte vectors per lane in a forward box
-constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor, per pass
-constexpr int kBwdHalves = GRK_BWD_HALVES;  // passes over a backward box
-constexpr unsigned kFwdBoxBytes = 32 * kFwdVec * 16;
-constexpr unsigned kBwdBoxBytes = 32 * kBwdVec * kBwdHalves * 16;
+constexpr int kBwdVec = 3;  // 16-byte vectors per lane and tensor in one backward pass
+
+template <class IO>
+struct Shape;
+template <>
+struct Shape<IoF32> {
+  static constexpr int kFwdVec = GRK_F32_FWD_VEC;        // vectors per lane in a forward box
+  static constexpr int kFwdStages = GRK_F32_FWD_STAGES;  // forward ring depth
+  static constexpr int kBwdHalves = GRK_F32_BWD_HALVES;  // passes over a backward box
+  static constexpr int kBwdStages = GRK_F32_BWD_STAGES;  // backward ring depth
+};
+template <>
+struct Shape<IoBF16> {
+  static constexpr int kFwdVec = GRK_BF16_FWD_VEC;
+  static constexpr int kFwdStages = GRK_BF16_FWD_STAGES;
+  static constexpr int kBwdHalves = GRK_BF16_BWD_HALVES;
+  static constexpr int kBwdStages = GRK_BF16_BWD_STAGES;
+};
+template <class IO>
+constexpr unsigned fwd_box_bytes() {
+  return 32u * Shape<IO>::kFwdVec * 16u;
+}
+template <class IO>
+constexpr unsigned bwd_box_bytes() {
+  return 32u * kBwdVec * Shape<IO>::kBwdHalves * 16u;
+}
+inline unsigned fwd_box_target(bool bf16) {
+  return bf16 ? fwd_box_bytes<IoBF16>() : fwd_box_bytes<IoF32>();
+}
+inline unsigned bwd_box_target(bool bf16) {
+  return bf16 ? bwd_box_bytes<IoBF16>() : bwd_box_bytes<IoF32>();
+}
 #ifndef GRK_BOXES_PER_UNIT
 #define GRK_BOXES_PER_UNIT 8
 #endif
@@ -374,20 +411,21 @@ template <class IO>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
+  using S_ = Shape<IO>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const WarpLayout L(geom.box_bytes, 1, kFwdStages);
+  const WarpLayout L(geom.box_bytes, 1, S_::kFwdStages);
   unsigned char* base = smem + warp * L.per_warp;
   float* cslot = reinterpret_cast<float*>(base + L.coef_off);
   const uint32_t full0 = smem_addr(base + L.bar_off);
-  const uint32_t empty0 = full0 + 8 * kFwdStages;
+  const uint32_t empty0 = full0 + 8 * S_::kFwdStages;
   const long long row_blocks = (geom.rows + geom.SCw - 1) / geom.SCw;
   const long long gw = (long long)blockIdx.x * kWarps + warp;
   const long long GW = (long long)gridDim.x * kWarps;
 
   if (lane == 0) {
-    for (int s = 0; s < kFwdStages; ++s) {
+    for (int s = 0; s < S_::kFwdStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
@@ -401,7 +439,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   ic.init(gw, GW, geom.n_g, geom.nbox);
   int iq = 0;
   auto issue = [&]() {
-    const int s = iq % kFwdStages;
+    const int s = iq % S_::kFwdStages;
     mbar_arrive_expect_tx(full0 + 8 * s, geom.box_bytes);
     tma_load_2d(smem_addr(base + s * L.stage), &mx, ic.mid * geom.dg + ic.lo * geom.bw,
                 (int)(ic.hi * geom.SCw), full0 + 8 * s);
@@ -409,10 +447,10 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     ++iq;
   };
   if (lane == 0)
-    for (int s = 0; s < kFwdStages && ic.hi < row_blocks; ++s) issue();
+    for (int s = 0; s < S_::kFwdStages && ic.hi < row_blocks; ++s) issue();
   __syncwarp();
 
-  LaneMap<IO, kFwdVec> lm;
+  LaneMap<IO, S_::kFwdVec> lm;
   lm.init(geom, lane, geom.d);
   Coef54 c;
   int cur_g = -1;
@@ -421,8 +459,8 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   Cursor3 cc;  // consumer cursor
   cc.init(gw, GW, geom.n_g, geom.nbox);
   for (; cc.hi < row_blocks; cc.next(), ++q) {
-    const int s = q % kFwdStages;
-    const uint32_t ph = (uint32_t)(q / kFwdStages) & 1;
+    const int s = q % S_::kFwdStages;
+    const uint32_t ph = (uint32_t)(q / S_::kFwdStages) & 1;
     if (!mbar_wait(full0 + 8 * s, ph)) {
       report(kErrFullWait);
       ok = false;
@@ -434,11 +472,11 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
       cur_g = g;
     }
     const uint4* buf = reinterpret_cast<const uint4*>(base + s * L.stage);
-    uint4 v[kFwdVec];
+    uint4 v[S_::kFwdVec];
 #pragma unroll
-    for (int it = 0; it < kFwdVec; ++it)
+    for (int it = 0; it < S_::kFwdVec; ++it)
       if (lm.row[it] < geom.SCw) v[it] = buf[lane + 32 * it];
-    // release the slot and refill it with the item kFwdStages ahead
+    // release the slot and refill it with the item S_::kFwdStages ahead
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(empty0 + 8 * s);
@@ -454,7 +492,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     const long long row0 = cc.hi * geom.SCw;
     typename IO::T* yo = y + row0 * geom.d + (g * geom.dg + cc.lo * geom.bw);
 #pragma unroll
-    for (int it = 0; it < kFwdVec; ++it) {
+    for (int it = 0; it < S_::kFwdVec; ++it) {
       if (row0 + lm.row[it] < geom.rows) {
         uint4 o;
         if constexpr (IO::kBytes == 2) {
@@ -479,7 +517,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   if (!ok && lane == 0) {
     // wind down: let every issued load land before the CTA's memory goes away
     for (int j = q; j < iq; ++j)
-      if (!mbar_wait(full0 + 8 * (j % kFwdStages), (uint32_t)(j / kFwdStages) & 1))
+      if (!mbar_wait(full0 + 8 * (j % S_::kFwdStages), (uint32_t)(j / S_::kFwdStages) & 1))
         report(kErrDrainWait);
   }
 }
@@ -503,19 +541,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
         typename IO::T* __restrict__ dx, const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
+  using S_ = Shape<IO>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const WarpLayout L(geom.box_bytes, 2, kBwdStages);
+  const WarpLayout L(geom.box_bytes, 2, S_::kBwdStages);
   unsigned char* base = smem + warp * L.per_warp;
   float* cslot = reinterpret_cast<float*>(base + L.coef_off);
   const uint32_t full0 = smem_addr(base + L.bar_off);
-  const uint32_t empty0 = full0 + 8 * kBwdStages;
+  const uint32_t empty0 = full0 + 8 * S_::kBwdStages;
   const long long gw = (long long)blockIdx.x * kWarps + warp;
   const long long GW = (long long)gridDim.x * kWarps;
 
   if (lane == 0) {
-    for (int s = 0; s < kBwdStages; ++s) {
+    for (int s = 0; s < S_::kBwdStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
@@ -534,7 +573,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   int irb = 0, ibx = 0, inrb = (iu.hi < geom.T) ? tile_row_blocks(geom, iu.hi) : 0;
   int iq = 0;
   auto issue = [&]() {
-    const int s = iq % kBwdStages;
+    const int s = iq % S_::kBwdStages;
     const int col = iu.lo * geom.dg + ibx * geom.bw;
     const int row = (int)(iu.hi * geom.S) + irb * geom.SCw;
     unsigned char* st = base + s * L.stage;
@@ -552,10 +591,10 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     }
   };
   if (lane == 0)
-    for (int s = 0; s < kBwdStages && iu.hi < geom.T; ++s) issue();
+    for (int s = 0; s < S_::kBwdStages && iu.hi < geom.T; ++s) issue();
   __syncwarp();
 
-  LaneMap<IO, kBwdVec * kBwdHalves> lm;
+  LaneMap<IO, kBwdVec * S_::kBwdHalves> lm;
   lm.init(geom, lane, geom.d);
   Coef54 c;
   int cur_g = -1;
@@ -577,8 +616,8 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     const long long rows_left = geom.rows - tile * geom.S;
     for (int rb = 0; rb < nrb && ok; ++rb) {
       for (int bx = 0; bx < geom.nbox; ++bx, ++q) {
-        const int s = q % kBwdStages;
-        const uint32_t ph = (uint32_t)(q / kBwdStages) & 1;
+        const int s = q % S_::kBwdStages;
+        const uint32_t ph = (uint32_t)(q / S_::kBwdStages) & 1;
         if (!mbar_wait(full0 + 8 * s, ph)) {
           report(kErrFullWait);
           ok = false;
@@ -589,7 +628,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         const int r0 = rb * geom.SCw;  // row of the box within the tile
         typename IO::T* dxo = dxt + (long long)r0 * geom.d + bx * geom.bw;
 #pragma unroll
-        for (int h = 0; h < kBwdHalves; ++h) {
+        for (int h = 0; h < S_::kBwdHalves; ++h) {
           uint4 xv[kBwdVec], gv[kBwdVec];
 #pragma unroll
           for (int it = 0; it < kBwdVec; ++it) {
@@ -602,7 +641,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
               gv[it] = make_uint4(0, 0, 0, 0);
             }
           }
-          if (h == kBwdHalves - 1) {
+          if (h == S_::kBwdHalves - 1) {
             // release the slot (every lane has read it) and refill it
             __syncwarp();
             if (lane == 0) {
@@ -668,7 +707,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   }
   if (!ok && lane == 0) {
     for (int j = q; j < iq; ++j)
-      if (!mbar_wait(full0 + 8 * (j % kBwdStages), (uint32_t)(j / kBwdStages) & 1))
+      if (!mbar_wait(full0 + 8 * (j % S_::kBwdStages), (uint32_t)(j / S_::kBwdStages) & 1))
         report(kErrDrainWait);
   }
 }
@@ -697,21 +736,28 @@ inline cudaError_t ensure_smem(unsigned bytes) {
 }
 
 // Shared memory of a launch: kWarps per-warp regions of the largest box.
-inline unsigned fwd_smem_bytes() { return kWarps * WarpLayout(kFwdBoxBytes, 1, kFwdStages).per_warp; }
-inline unsigned bwd_smem_bytes() { return kWarps * WarpLayout(kBwdBoxBytes, 2, kBwdStages).per_warp; }
+template <class IO>
+inline unsigned fwd_smem_bytes() {
+  return kWarps * WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages).per_warp;
+}
+template <class IO>
+inline unsigned bwd_smem_bytes() {
+  return kWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp;
+}
 
 inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx, void* y,
                                   const float* a, const float* b, int sms, cudaStream_t st) {
-  if (g.box_bytes > kFwdBoxBytes) return cudaErrorInvalidValue;
-  const unsigned smem = fwd_smem_bytes();
+  if (g.box_bytes > fwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long items = ((g.rows + g.SCw - 1) / g.SCw) * g.n_g * g.nbox;
   long long grid = sms;
   if (grid * kWarps > items) grid = (items + kWarps - 1) / kWarps;
   cudaError_t e;
   if (bf16) {
+    const unsigned smem = fwd_smem_bytes<IoBF16>();
     if ((e = ensure_smem<IoBF16, false>(smem)) != cudaSuccess) return e;
     fwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoBF16::T*)y, a, b, g);
   } else {
+    const unsigned smem = fwd_smem_bytes<IoF32>();
     if ((e = ensure_smem<IoF32, false>(smem)) != cudaSuccess) return e;
     fwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoF32::T*)y, a, b, g);
   }
@@ -721,17 +767,18 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
 inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
                                   const CUtensorMap& mdy, void* dx, const float* a,
                                   const float* b, float* ws, int sms, cudaStream_t st) {
-  if (g.box_bytes > kBwdBoxBytes) return cudaErrorInvalidValue;
-  const unsigned smem = bwd_smem_bytes();
+  if (g.box_bytes > bwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long units = g.T * g.n_g;
   long long grid = sms;
   if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
   cudaError_t e;
   if (bf16) {
+    const unsigned smem = bwd_smem_bytes<IoBF16>();
     if ((e = ensure_smem<IoBF16, true>(smem)) != cudaSuccess) return e;
     bwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, mdy, (IoBF16::T*)dx, a, b,
                                                                 ws, g);
   } else {
+    const unsigned smem = bwd_smem_bytes<IoF32>();
     if ((e = ensure_smem<IoF32, true>(smem)) != cudaSuccess) return e;
     bwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, mdy, (IoF32::T*)dx, a, b, ws,
                                                                g);

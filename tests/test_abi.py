@@ -45,8 +45,9 @@ def test_workspace_bytes():
     # KAT-B: d_g = 384 bf16 -> backward boxes of 8 rows x 192 channels (3 KiB), 2 per
     # group row, 8 boxes per unit -> 32 rows per tile, 3152 tiles
     assert grk.grkan_backward_workspace_bytes(512, 197, 3072, 8, 5, 4, grk.BF16) == 3152 * 8 * 10 * 4
-    # KAT-T: d_g = 96 f32 -> boxes of 8 rows x 96 channels -> 64 rows per tile, 3152 tiles
-    assert grk.grkan_backward_workspace_bytes(1024, 197, 768, 8, 5, 4, grk.F32) == 3152 * 8 * 10 * 4
+    # KAT-T: d_g = 96 f32 -> boxes of 4 rows x 96 channels (1.5 KiB) -> 32 rows per
+    # tile, 6304 tiles
+    assert grk.grkan_backward_workspace_bytes(1024, 197, 768, 8, 5, 4, grk.F32) == 6304 * 8 * 10 * 4
     assert grk.grkan_backward_workspace_bytes(0, 197, 768, 8, 5, 4, grk.F32) == 0
     assert grk.grkan_backward_workspace_bytes(2, 3, 10, 3, 5, 4, grk.F32) == 0  # d % n_g != 0
     assert grk.grkan_backward_workspace_bytes(2, 3, 12, 3, 9, 4, grk.F32) == 0  # degree

@@ -69,8 +69,9 @@ def test_noalloc_matches_workspace_entry_point_call_after_call():
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():
-    need = grk.grkan_backward_workspace_bytes(2048, 197, 3072, 8, 5, 4, grk.BF16)
+    B = 16384  # a KAT-B-width activation 32 times the size of the workload's batch
+    need = grk.grkan_backward_workspace_bytes(B, 197, 3072, 8, 5, 4, grk.BF16)
     assert need > grk.NOALLOC_WORKSPACE_BYTES
     x = torch.empty(8, device="cuda")
-    st = grk.grkan_backward_noalloc(x, x, x, x, x, x, x, 2048, 197, 3072, 8, 5, 4, grk.BF16)
+    st = grk.grkan_backward_noalloc(x, x, x, x, x, x, x, B, 197, 3072, 8, 5, 4, grk.BF16)
     assert st == 5  # GRKAN_ERR_WORKSPACE, nothing launched
