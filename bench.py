@@ -303,20 +303,27 @@ def main():
     ms_step = ms_total / args.steps
     value = E * world / (ms_step * 1e-3)
 
-    # end to end through the same ABI calls, host (pinned) buffers in and out
+    # end to end through the C ABI's host-buffer entry point: pinned inputs in,
+    # y, dx and dA/dB out, copies inside the timed region (chunks streamed over
+    # three streams so that copies in, kernels and copies out overlap)
     y_h = torch.empty_like(x_h, pin_memory=True)
     dx_h = torch.empty_like(x_h, pin_memory=True)
-    dA_h = torch.empty_like(dA, device="cpu", pin_memory=True)
-    dB_h = torch.empty_like(dB, device="cpu", pin_memory=True)
+    dA_h = torch.empty(dA.shape, dtype=torch.float32, pin_memory=True)
+    dB_h = torch.empty(dB.shape, dtype=torch.float32, pin_memory=True)
+    del x, dy, y, dx  # the host path stages its own chunks
+    torch.cuda.empty_cache()
+    sneed = grk.grkan_step_host_scratch_bytes(B, N, d, n_g, m, n, dt, 0)
+    scratch = torch.empty(sneed, dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        x.copy_(x_h, non_blocking=True)
-        dy.copy_(dy_h, non_blocking=True)
-        step()
-        y_h.copy_(y, non_blocking=True)
-        dx_h.copy_(dx, non_blocking=True)
-        dA_h.copy_(dA, non_blocking=True)
-        dB_h.copy_(dB, non_blocking=True)
+        check(grk.grkan_step_host(x_h, dy_h, a, b, y_h, dx_h, dA_h, dB_h, B, N, d, n_g, m, n, dt,
+                                  scratch, sneed, 0, sp), "step_host")
+        if world > 1:  # the data-parallel exchange of this rank's gradients
+            stream.synchronize()
+            s64 = torch.from_numpy(np.concatenate([dA_h.numpy(), dB_h.numpy()], 1)).to(
+                dev, torch.float64)
+            g = all_gather_sums(s64)
+            check(grk.grkan_merge_ranks(g, world, dA, dB, n_g, m, n, sp), "merge_ranks")
 
     for _ in range(min(2, args.e2e_steps)):
         e2e_step()
@@ -369,7 +376,8 @@ def main():
         },
         "e2e": {"value": E * world / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": 2 * nbytes,
-                "d2h_bytes_per_step": 2 * nbytes + (n_g * K) * 4, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": 2 * nbytes + (n_g * K) * 4, "ms_per_step": e2e_ms,
+                "api": "grkan_step_host (x, dy in; y, dx, dA, dB out; pinned host buffers)"},
         "gpu_launches": args.steps * (3 + (1 if world > 1 else 0)),
         "clocks": clocks,
         "device_error": derr,

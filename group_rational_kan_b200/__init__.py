@@ -17,6 +17,7 @@ __all__ = [
     "grkan_forward", "grkan_forward_ex", "grkan_backward", "grkan_backward_ex",
     "grkan_backward_partials", "grkan_backward_merge", "grkan_backward_workspace_bytes",
     "grkan_merge_ranks", "grkan_backward_noalloc", "NOALLOC_WORKSPACE_BYTES",
+    "grkan_step_host", "grkan_step_host_scratch_bytes",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
     "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
 ]
@@ -64,6 +65,9 @@ def _load():
         "grkan_backward_merge": (S, [P, SZ, P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int,
                                      P]),
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
+        "grkan_step_host_scratch_bytes": (SZ, [I64, I64, I64, I32, I32, I32, ctypes.c_int, I64]),
+        "grkan_step_host": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
+                                ctypes.c_int, P, SZ, I64, P]),
         "grkan_backward_noalloc": (S, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                        ctypes.c_int, P]),
         "grkan_forward_path": (I32, [P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int, U32]),
@@ -164,6 +168,19 @@ def grkan_backward_noalloc(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, s
     callers that cannot allocate device memory per call)."""
     return lib().grkan_backward_noalloc(_ptr(x), _ptr(dy), _ptr(a), _ptr(b), _ptr(dx), _ptr(dA),
                                         _ptr(dB), B, N, d, n_g, m, n, dtype, _stream(stream))
+
+
+def grkan_step_host_scratch_bytes(B, N, d, n_g, m, n, dtype, chunk_rows=0):
+    return lib().grkan_step_host_scratch_bytes(B, N, d, n_g, m, n, dtype, chunk_rows)
+
+
+def grkan_step_host(x_host, dy_host, a, b, y_host, dx_host, dA_host, dB_host, B, N, d, n_g, m, n,
+                    dtype, scratch, scratch_bytes, chunk_rows=0, stream=None):
+    """Forward + backward of host tensors (pinned torch CPU tensors or raw host
+    pointers) streamed through device scratch; dA_host / dB_host are host."""
+    return lib().grkan_step_host(_ptr(x_host), _ptr(dy_host), _ptr(a), _ptr(b), _ptr(y_host),
+                                 _ptr(dx_host), _ptr(dA_host), _ptr(dB_host), B, N, d, n_g, m, n,
+                                 dtype, _ptr(scratch), scratch_bytes, chunk_rows, _stream(stream))
 
 
 def grkan_forward_path(x, y, B, N, d, n_g, m, n, dtype, flags=0):

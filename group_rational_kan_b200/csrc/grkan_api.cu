@@ -48,24 +48,24 @@ struct Box {
   unsigned bytes = 0;
 };
 
-// The largest box at most `target` bytes: width the largest divisor of d_g
-// that is at most 256 elements, a whole number of 16-byte vectors and fits,
-// height as many rows as fit (at most 256).
+// The box of at most `target` bytes that holds the most data: width a divisor
+// of d_g of at most 256 elements and a whole number of 16-byte vectors, height
+// as many rows as fit (at most 256); among equally full boxes the widest.
 Box choose_box(long long dg, int es, unsigned target) {
   Box b;
   if (dg <= 0) return b;
   for (long long w = dg < 256 ? dg : 256; w >= 1; --w) {
-    if (dg % w == 0 && (w * es) % 16 == 0 && (unsigned)(w * es) <= target) {
+    if (dg % w != 0 || (w * es) % 16 != 0 || (unsigned)(w * es) > target) continue;
+    long long rows = target / (unsigned)(w * es);
+    if (rows > kMaxBoxRows) rows = kMaxBoxRows;
+    const unsigned bytes = (unsigned)(rows * w * es);
+    if (bytes > b.bytes) {
       b.bw = (int)w;
-      break;
+      b.scw = (int)rows;
+      b.nbox = (int)(dg / w);
+      b.bytes = bytes;
     }
   }
-  if (b.bw == 0) return b;
-  long long rows = target / (unsigned)(b.bw * es);
-  if (rows > kMaxBoxRows) rows = kMaxBoxRows;
-  b.scw = (int)rows;
-  b.nbox = (int)(dg / b.bw);
-  b.bytes = (unsigned)(b.scw * b.bw * es);
   return b;
 }
 
@@ -156,11 +156,12 @@ cudaError_t launch_generic_fwd(const Plan& p, const void* x, void* y, const floa
 
 template <class IO>
 cudaError_t launch_generic_bwd(const Plan& p, const void* x, const void* dy, void* dx,
-                               const float* a, const float* b, float* ws, cudaStream_t st) {
+                               const float* a, const float* b, float* ws, long long ws_T,
+                               long long tile0, cudaStream_t st) {
   const long long units = p.T * p.n_g;
   grk::bwd_generic<IO, GRKAN_MAX_M, GRKAN_MAX_N><<<(unsigned)units, grk::kGenericThreads, 0, st>>>(
       (const typename IO::T*)x, (const typename IO::T*)dy, (typename IO::T*)dx, a, b, ws, p.rows,
-      p.d, (int)p.dg, p.n_g, p.m, p.n, (int)p.S, p.T);
+      p.d, (int)p.dg, p.n_g, p.m, p.n, (int)p.S, ws_T, tile0);
   return cudaGetLastError();
 }
 
@@ -245,6 +246,8 @@ grk::TmaGeom make_geom(const Plan& p, const Box& bx) {
   grk::TmaGeom g;
   g.rows = p.rows;
   g.T = p.T;
+  g.ws_T = p.T;
+  g.ws_tile0 = 0;
   g.d = p.d;
   g.S = p.S;
   g.dg = (int)p.dg;
@@ -280,10 +283,13 @@ grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float
 }
 
 grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx,
-                              const float* a, const float* b, float* ws, cudaStream_t st) {
+                              const float* a, const float* b, float* ws, long long ws_T,
+                              long long tile0, cudaStream_t st) {
   CUtensorMap mx, mdy;
   if (!make_map(&mx, x, p, p.bbox) || !make_map(&mdy, dy, p, p.bbox)) return GRKAN_ERR_CUDA;
-  const grk::TmaGeom geom = make_geom(p, p.bbox);
+  grk::TmaGeom geom = make_geom(p, p.bbox);
+  geom.ws_T = ws_T;
+  geom.ws_tile0 = tile0;
   cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, dx, a, b, ws,
                                       sm_count(), st);
   return cuda_status(e, "backward (TMA) launch");
@@ -315,6 +321,21 @@ grkan_status_t do_forward(const void* x, void* y, const float* a, const float* b
   return cuda_status(e, "forward (generic) launch");
 }
 
+// Stage 1 into the workspace; the partials of this call's tiles go to tiles
+// [tile0, tile0 + p.T) of a workspace laid out for ws_T tiles (a whole tensor).
+grkan_status_t do_partials_at(const Plan& p, const void* x, const void* dy, const float* a,
+                              const float* b, void* dx, void* ws, long long ws_T, long long tile0,
+                              uint32_t flags, cudaStream_t st) {
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  if (choose_bwd_path(p, x, dy, dx, flags) == 1)
+    return launch_tma_bwd(p, x, dy, dx, a, b, (float*)ws, ws_T, tile0, st);
+  cudaError_t e =
+      (p.dtype == GRKAN_F32)
+          ? launch_generic_bwd<grk::IoF32>(p, x, dy, dx, a, b, (float*)ws, ws_T, tile0, st)
+          : launch_generic_bwd<grk::IoBF16>(p, x, dy, dx, a, b, (float*)ws, ws_T, tile0, st);
+  return cuda_status(e, "backward (generic) launch");
+}
+
 grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const float* a,
                            const float* b, void* dx, void* ws, size_t ws_bytes, uint32_t flags,
                            cudaStream_t st) {
@@ -327,14 +348,7 @@ grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const f
   if (overlaps(ws, p.ws_bytes, x, bytes) || overlaps(ws, p.ws_bytes, dy, bytes) ||
       overlaps(ws, p.ws_bytes, dx, bytes))
     return GRKAN_ERR_ALIAS;
-  if (!is_sm100()) return GRKAN_ERR_DEVICE;
-  if (choose_bwd_path(p, x, dy, dx, flags) == 1)
-    return launch_tma_bwd(p, x, dy, dx, a, b, (float*)ws, st);
-  cudaError_t e =
-      (p.dtype == GRKAN_F32)
-          ? launch_generic_bwd<grk::IoF32>(p, x, dy, dx, a, b, (float*)ws, st)
-          : launch_generic_bwd<grk::IoBF16>(p, x, dy, dx, a, b, (float*)ws, st);
-  return cuda_status(e, "backward (generic) launch");
+  return do_partials_at(p, x, dy, a, b, dx, ws, p.T, 0, flags, st);
 }
 
 grkan_status_t do_merge(const Plan& p, const void* ws, size_t ws_bytes, float* dA, float* dB,
@@ -371,6 +385,82 @@ grkan_status_t noalloc_workspace(void** out) {
   }
   *out = g_noalloc_ptr[dev];
   return GRKAN_OK;
+}
+
+// --- host-buffer step: row chunks streamed through device staging -------------------
+//
+// Three streams per device (created on first use and kept): host-to-device
+// copies, kernels, device-to-host copies. Chunk c uses staging slot c % kSlots;
+// a slot is refilled only after its previous results have left the device.
+// Chunks are whole row tiles, so the partial sums land exactly where a single
+// grkan_backward would put them and the merged gradients are the same bits.
+
+constexpr int kSlots = 3;
+constexpr long long kChunkTarget = 32LL << 20;  // bytes of one tensor chunk
+
+struct HostPipe {
+  cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr, comp_done = nullptr, out_done = nullptr;
+  cudaEvent_t in[kSlots] = {}, comp[kSlots] = {}, out[kSlots] = {};
+  bool ready = false;
+};
+
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kMaxDevices];
+
+grkan_status_t pipe_for_device(int dev, HostPipe** out) {
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    const unsigned fl = cudaStreamNonBlocking;
+    grkan_status_t s = cuda_status(cudaStreamCreateWithFlags(&hp.s_in, fl), "cudaStreamCreate");
+    if (s == GRKAN_OK) s = cuda_status(cudaStreamCreateWithFlags(&hp.s_comp, fl), "cudaStreamCreate");
+    if (s == GRKAN_OK) s = cuda_status(cudaStreamCreateWithFlags(&hp.s_out, fl), "cudaStreamCreate");
+    cudaEvent_t* evs[] = {&hp.start, &hp.comp_done, &hp.out_done};
+    for (cudaEvent_t* e : evs)
+      if (s == GRKAN_OK)
+        s = cuda_status(cudaEventCreateWithFlags(e, cudaEventDisableTiming), "cudaEventCreate");
+    for (int i = 0; i < kSlots && s == GRKAN_OK; ++i) {
+      s = cuda_status(cudaEventCreateWithFlags(&hp.in[i], cudaEventDisableTiming), "cudaEventCreate");
+      if (s == GRKAN_OK)
+        s = cuda_status(cudaEventCreateWithFlags(&hp.comp[i], cudaEventDisableTiming),
+                        "cudaEventCreate");
+      if (s == GRKAN_OK)
+        s = cuda_status(cudaEventCreateWithFlags(&hp.out[i], cudaEventDisableTiming),
+                        "cudaEventCreate");
+    }
+    if (s != GRKAN_OK) return s;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return GRKAN_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Rows per chunk: a whole number of row tiles, about kChunkTarget bytes of one
+// tensor (or what the caller asked for, rounded up to whole tiles).
+long long chunk_rows_for(const Plan& p, long long want) {
+  long long rows = want > 0 ? want : kChunkTarget / (p.d * p.es > 0 ? p.d * p.es : 1);
+  if (rows < p.S) rows = p.S;
+  rows = (rows + p.S - 1) / p.S * p.S;
+  if (rows > p.rows) rows = (p.rows + p.S - 1) / p.S * p.S;
+  return rows < 1 ? 1 : rows;
+}
+
+struct StagingLayout {
+  long long chunk_rows = 0;
+  size_t tensor = 0;  // bytes of one chunk buffer
+  size_t ws_off = 0, grad_off = 0, total = 0;
+};
+
+StagingLayout staging_layout(const Plan& p, long long want_rows) {
+  StagingLayout L;
+  L.chunk_rows = chunk_rows_for(p, want_rows);
+  L.tensor = align256((size_t)L.chunk_rows * (size_t)p.d * (size_t)p.es);
+  L.ws_off = (size_t)kSlots * 4 * L.tensor;  // per slot: x, dy, y, dx
+  L.grad_off = L.ws_off + align256(p.ws_bytes);
+  L.total = L.grad_off + align256((size_t)p.n_g * (size_t)p.K * sizeof(float));
+  return L;
 }
 
 }  // namespace
@@ -482,6 +572,115 @@ grkan_status_t grkan_backward_noalloc(const void* x, const void* dy, const float
     if (s != GRKAN_OK) return s;
   }
   return do_merge(p, ws, GRKAN_NOALLOC_WORKSPACE_BYTES, dA, dB, nullptr, st);
+}
+
+size_t grkan_step_host_scratch_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
+                                     int32_t n, grkan_dtype_t dtype, int64_t chunk_rows) {
+  Plan p;
+  if (make_plan(B, N, d, n_g, m, n, dtype, &p) != GRKAN_OK) return 0;
+  if (p.rows == 0 || p.d == 0) return 256;
+  return staging_layout(p, chunk_rows).total;
+}
+
+grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const float* a,
+                               const float* b, void* y_host, void* dx_host, float* dA_host,
+                               float* dB_host, int64_t B, int64_t N, int64_t d, int32_t n_g,
+                               int32_t m, int32_t n, grkan_dtype_t dtype, void* scratch,
+                               size_t scratch_bytes, int64_t chunk_rows, void* stream) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (!dA_host || (p.n > 0 && !dB_host)) return GRKAN_ERR_NULL;
+  if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+  const bool empty = p.rows == 0 || p.d == 0;
+  if (!empty && (!x_host || !dy_host || !y_host || !dx_host)) return GRKAN_ERR_NULL;
+  const StagingLayout L = empty ? StagingLayout() : staging_layout(p, chunk_rows);
+  const size_t need = empty ? 256 : L.total;
+  if (!scratch || scratch_bytes < need || ((uintptr_t)scratch & 255u)) return GRKAN_ERR_WORKSPACE;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  int dev = 0;
+  if ((s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice")) != GRKAN_OK) return s;
+  if (dev < 0 || dev >= kMaxDevices) return GRKAN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe* hp = nullptr;
+  if ((s = pipe_for_device(dev, &hp)) != GRKAN_OK) return s;
+  cudaStream_t caller = (cudaStream_t)stream;
+  unsigned char* base = (unsigned char*)scratch;
+  float* ws = (float*)(base + L.ws_off);
+  float* dA = (float*)(base + L.grad_off);
+  float* dB = dA + (size_t)p.n_g * (p.m + 1);
+  const size_t ka = (size_t)p.n_g * (p.m + 1) * sizeof(float);
+  const size_t kb = (size_t)p.n_g * p.n * sizeof(float);
+
+#define GRK_TRY(expr, what)                                   \
+  do {                                                        \
+    if ((s = cuda_status((expr), what)) != GRKAN_OK) return s; \
+  } while (0)
+
+  // everything issued before on the caller's stream happens first
+  GRK_TRY(cudaEventRecord(hp->start, caller), "cudaEventRecord");
+  GRK_TRY(cudaStreamWaitEvent(hp->s_in, hp->start, 0), "cudaStreamWaitEvent");
+  GRK_TRY(cudaStreamWaitEvent(hp->s_comp, hp->start, 0), "cudaStreamWaitEvent");
+  GRK_TRY(cudaStreamWaitEvent(hp->s_out, hp->start, 0), "cudaStreamWaitEvent");
+  if (empty) {
+    s = do_merge(p, ws, 0, dA, dB, nullptr, hp->s_comp);
+    if (s != GRKAN_OK) return s;
+  } else {
+    const long long nchunks = (p.rows + L.chunk_rows - 1) / L.chunk_rows;
+    const size_t row_bytes = (size_t)p.d * (size_t)p.es;
+    for (long long c = 0; c < nchunks; ++c) {
+      const int slot = (int)(c % kSlots);
+      const long long r0 = c * L.chunk_rows;
+      const long long rows = (p.rows - r0) < L.chunk_rows ? (p.rows - r0) : L.chunk_rows;
+      const size_t bytes = (size_t)rows * row_bytes;
+      const size_t off = (size_t)r0 * row_bytes;
+      unsigned char* sx = base + (size_t)slot * 4 * L.tensor;
+      unsigned char* sdy = sx + L.tensor;
+      unsigned char* sy = sdy + L.tensor;
+      unsigned char* sdx = sy + L.tensor;
+      // inputs in, once the slot's previous outputs have left
+      if (c >= kSlots) GRK_TRY(cudaStreamWaitEvent(hp->s_in, hp->out[slot], 0), "cudaStreamWaitEvent");
+      GRK_TRY(cudaMemcpyAsync(sx, (const unsigned char*)x_host + off, bytes,
+                              cudaMemcpyHostToDevice, hp->s_in), "cudaMemcpyAsync");
+      GRK_TRY(cudaMemcpyAsync(sdy, (const unsigned char*)dy_host + off, bytes,
+                              cudaMemcpyHostToDevice, hp->s_in), "cudaMemcpyAsync");
+      GRK_TRY(cudaEventRecord(hp->in[slot], hp->s_in), "cudaEventRecord");
+      // forward and backward of the chunk; its tiles go to their place in ws
+      GRK_TRY(cudaStreamWaitEvent(hp->s_comp, hp->in[slot], 0), "cudaStreamWaitEvent");
+      Plan pc;
+      if ((s = make_plan(rows, 1, p.d, p.n_g, p.m, p.n, p.dtype, &pc)) != GRKAN_OK) return s;
+      if (choose_fwd_path(pc, sx, sy, 0) == 1) {
+        s = launch_tma_fwd(pc, sx, sy, a, b, hp->s_comp);
+      } else {
+        cudaError_t e = (p.dtype == GRKAN_F32)
+                            ? launch_generic_fwd<grk::IoF32>(pc, sx, sy, a, b, hp->s_comp)
+                            : launch_generic_fwd<grk::IoBF16>(pc, sx, sy, a, b, hp->s_comp);
+        s = cuda_status(e, "forward (generic) launch");
+      }
+      if (s != GRKAN_OK) return s;
+      s = do_partials_at(pc, sx, sdy, a, b, sdx, ws, p.T, r0 / p.S, 0u, hp->s_comp);
+      if (s != GRKAN_OK) return s;
+      GRK_TRY(cudaEventRecord(hp->comp[slot], hp->s_comp), "cudaEventRecord");
+      // outputs out
+      GRK_TRY(cudaStreamWaitEvent(hp->s_out, hp->comp[slot], 0), "cudaStreamWaitEvent");
+      GRK_TRY(cudaMemcpyAsync((unsigned char*)y_host + off, sy, bytes, cudaMemcpyDeviceToHost,
+                              hp->s_out), "cudaMemcpyAsync");
+      GRK_TRY(cudaMemcpyAsync((unsigned char*)dx_host + off, sdx, bytes, cudaMemcpyDeviceToHost,
+                              hp->s_out), "cudaMemcpyAsync");
+      GRK_TRY(cudaEventRecord(hp->out[slot], hp->s_out), "cudaEventRecord");
+    }
+    s = do_merge(p, ws, p.ws_bytes, dA, dB, nullptr, hp->s_comp);
+    if (s != GRKAN_OK) return s;
+  }
+  GRK_TRY(cudaMemcpyAsync(dA_host, dA, ka, cudaMemcpyDeviceToHost, hp->s_comp), "cudaMemcpyAsync");
+  if (kb) GRK_TRY(cudaMemcpyAsync(dB_host, dB, kb, cudaMemcpyDeviceToHost, hp->s_comp), "cudaMemcpyAsync");
+  GRK_TRY(cudaEventRecord(hp->comp_done, hp->s_comp), "cudaEventRecord");
+  GRK_TRY(cudaEventRecord(hp->out_done, hp->s_out), "cudaEventRecord");
+  // the caller's stream continues after both
+  GRK_TRY(cudaStreamWaitEvent(caller, hp->comp_done, 0), "cudaStreamWaitEvent");
+  GRK_TRY(cudaStreamWaitEvent(caller, hp->out_done, 0), "cudaStreamWaitEvent");
+#undef GRK_TRY
+  return GRKAN_OK;
 }
 
 int32_t grkan_forward_path(const void* x, const void* y, int64_t B, int64_t N, int64_t d,

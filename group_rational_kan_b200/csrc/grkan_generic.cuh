@@ -37,12 +37,13 @@ fwd_generic(const typename IO::T* x, typename IO::T* y, const float* __restrict_
   }
 }
 
-// Partial sums of one unit -> ws[(g*K + k) * T + tile], K = m + 1 + n.
+// Partial sums of one unit -> ws[(g*K + k) * ws_T + tile0 + tile], K = m + 1 + n.
 template <class IO, int MM, int NM>
 __global__ void __launch_bounds__(kGenericThreads)
 bwd_generic(const typename IO::T* x, const typename IO::T* dy, typename IO::T* dx,
             const float* __restrict__ a, const float* __restrict__ b, float* __restrict__ ws,
-            long long rows, long long d, int dg, int n_g, int m, int n, int S, long long T) {
+            long long rows, long long d, int dg, int n_g, int m, int n, int S, long long ws_T,
+            long long tile0) {
   __shared__ float red[kGenericThreads / 32][MM + 1 + NM];
   const long long unit = blockIdx.x;
   const long long tile = unit / n_g;
@@ -92,7 +93,7 @@ bwd_generic(const typename IO::T* x, const typename IO::T* dy, typename IO::T* d
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < kGenericThreads / 32; ++w) s += red[w][slot];
-    ws[((long long)g * K + k) * T + tile] = s;
+    ws[((long long)g * K + k) * ws_T + tile0 + tile] = s;
   }
 }
 

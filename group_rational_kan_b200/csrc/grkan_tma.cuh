@@ -33,6 +33,8 @@ namespace grk {
 struct TmaGeom {
   long long rows;       // B * N
   long long T;          // row tiles (units per group)
+  long long ws_T;       // workspace stride between coefficients (tiles of the whole tensor)
+  long long ws_tile0;   // workspace tile of this call's first tile
   long long d;          // channels (row length)
   long long S;          // rows per tile
   int dg;               // channels per group
@@ -526,7 +528,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
 // Units (tile, g) (tile = S rows) are taken by warp gw of the grid as unit
 // gw, gw + total warps, ... in tile-major order; a unit's boxes are its row
 // blocks (SCw rows) times the group's column boxes. The partial sum of unit
-// (tile, g), coefficient k goes to ws[(g * 10 + k) * T + tile].
+// (tile, g), coefficient k goes to ws[(g * 10 + k) * ws_T + ws_tile0 + tile].
 
 
 // Row blocks of tile `tile`: ceil(min(S, rows - tile * S) / SCw).
@@ -703,7 +705,8 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     warp_sum10(v, lane);
     // after the exchange lane l holds the sum of coefficient (l >> 1) & 15
     const int k = (lane >> 1) & 15;
-    if ((lane & 1) == 0 && k < 10) ws[((long long)g * 10 + k) * geom.T + tile] = v[0];
+    if ((lane & 1) == 0 && k < 10)
+      ws[((long long)g * 10 + k) * geom.ws_T + geom.ws_tile0 + tile] = v[0];
   }
   if (!ok && lane == 0) {
     for (int j = q; j < iq; ++j)

@@ -166,6 +166,31 @@ GRKAN_API grkan_status_t grkan_backward_noalloc(const void* x, const void* dy, c
                                                 int32_t m, int32_t n, grkan_dtype_t dtype,
                                                 void* stream);
 
+/* One forward + backward step on HOST-resident tensors. x_host, dy_host (in) and
+ * y_host, dx_host (out) are host pointers to row-major (B, N, d) tensors (page-
+ * locked memory lets the copies overlap; pageable memory works but serialises);
+ * dA_host, dB_host receive the coefficient gradients (host pointers). a and b
+ * are device pointers, as everywhere. The rows stream through `scratch`, a
+ * device buffer of at least grkan_step_host_scratch_bytes(...) bytes (256-byte
+ * aligned, owned by the caller), in chunks of about 32 MiB per tensor (or
+ * chunk_rows rows, rounded up to whole reduction tiles) on three internal
+ * streams, so that the host-to-device copies, the kernels and the
+ * device-to-host copies of consecutive chunks overlap. The result is the same,
+ * bit for bit, as grkan_forward + grkan_backward on device copies of the same
+ * data. Asynchronous with respect to the host: the outputs are complete once
+ * `stream` reaches the point of the call. The first call on a device creates
+ * three streams and a few events that live until the process exits; calls are
+ * serialised per device while they enqueue. */
+GRKAN_API size_t grkan_step_host_scratch_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g,
+                                               int32_t m, int32_t n, grkan_dtype_t dtype,
+                                               int64_t chunk_rows);
+GRKAN_API grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const float* a,
+                                         const float* b, void* y_host, void* dx_host,
+                                         float* dA_host, float* dB_host, int64_t B, int64_t N,
+                                         int64_t d, int32_t n_g, int32_t m, int32_t n,
+                                         grkan_dtype_t dtype, void* scratch, size_t scratch_bytes,
+                                         int64_t chunk_rows, void* stream);
+
 /* Which kernels a call with these arguments would run: 1 = TMA-pipelined
  * persistent kernels, 0 = generic grid-stride kernels, < 0 = invalid arguments
  * (the negated status). x, y are only inspected for alignment. */
