@@ -48,25 +48,26 @@ struct Box {
   unsigned bytes = 0;
 };
 
-// The box of at most `target` bytes that holds the most data: width a divisor
-// of d_g of at most 256 elements and a whole number of 16-byte vectors, height
-// as many rows as fit (at most 256); among equally full boxes the widest.
+// The TMA box for a group: width a divisor of d_g of at most 256 elements and a
+// whole number of 16-byte vectors, height as many rows as fit in `target` bytes
+// (at most 256). Wide rows stream better, so the widest box that fills at least
+// three quarters of the target wins; if none does, the fullest box.
 Box choose_box(long long dg, int es, unsigned target) {
-  Box b;
-  if (dg <= 0) return b;
+  Box wide, full;
+  if (dg <= 0) return wide;
   for (long long w = dg < 256 ? dg : 256; w >= 1; --w) {
     if (dg % w != 0 || (w * es) % 16 != 0 || (unsigned)(w * es) > target) continue;
     long long rows = target / (unsigned)(w * es);
     if (rows > kMaxBoxRows) rows = kMaxBoxRows;
-    const unsigned bytes = (unsigned)(rows * w * es);
-    if (bytes > b.bytes) {
-      b.bw = (int)w;
-      b.scw = (int)rows;
-      b.nbox = (int)(dg / w);
-      b.bytes = bytes;
-    }
+    Box b;
+    b.bw = (int)w;
+    b.scw = (int)rows;
+    b.nbox = (int)(dg / w);
+    b.bytes = (unsigned)(rows * w * es);
+    if (wide.bw == 0 && 4ull * b.bytes >= 3ull * target) wide = b;
+    if (b.bytes > full.bytes) full = b;
   }
-  return b;
+  return wide.bw ? wide : full;
 }
 
 struct Plan {
