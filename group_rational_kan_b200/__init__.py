@@ -17,7 +17,8 @@ __all__ = [
     "grkan_forward", "grkan_forward_ex", "grkan_backward", "grkan_backward_ex",
     "grkan_backward_partials", "grkan_backward_merge", "grkan_backward_workspace_bytes",
     "grkan_merge_ranks", "grkan_backward_noalloc", "NOALLOC_WORKSPACE_BYTES",
-    "grkan_step_host", "grkan_step_host_scratch_bytes",
+    "grkan_step_host", "grkan_step_host_scratch_bytes", "grkan_forward_backward",
+    "forward_backward",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
     "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
 ]
@@ -65,6 +66,8 @@ def _load():
         "grkan_backward_merge": (S, [P, SZ, P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int,
                                      P]),
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
+        "grkan_forward_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
+                                       ctypes.c_int, P, SZ, U32, P]),
         "grkan_step_host_scratch_bytes": (SZ, [I64, I64, I64, I32, I32, I32, ctypes.c_int, I64]),
         "grkan_step_host": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                 ctypes.c_int, P, SZ, I64, P]),
@@ -168,6 +171,13 @@ def grkan_backward_noalloc(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, s
     callers that cannot allocate device memory per call)."""
     return lib().grkan_backward_noalloc(_ptr(x), _ptr(dy), _ptr(a), _ptr(b), _ptr(dx), _ptr(dA),
                                         _ptr(dB), B, N, d, n_g, m, n, dtype, _stream(stream))
+
+
+def grkan_forward_backward(x, dy, a, b, y, dx, dA, dB, B, N, d, n_g, m, n, dtype, workspace,
+                           workspace_bytes, flags=0, stream=None):
+    return lib().grkan_forward_backward(_ptr(x), _ptr(dy), _ptr(a), _ptr(b), _ptr(y), _ptr(dx),
+                                        _ptr(dA), _ptr(dB), B, N, d, n_g, m, n, dtype,
+                                        _ptr(workspace), workspace_bytes, flags, _stream(stream))
 
 
 def grkan_step_host_scratch_bytes(B, N, d, n_g, m, n, dtype, chunk_rows=0):
@@ -283,3 +293,19 @@ def backward(x, dy, a, b, n_g, dx=None, dA=None, dB=None, workspace=None, flags=
                              workspace.numel() * workspace.element_size(), flags, stream),
            "grkan_backward")
     return dx, dA, dB
+
+
+def forward_backward(x, dy, a, b, n_g, flags=0, stream=None):
+    """(y, dx, dA, dB) in one pass (recompute mode)."""
+    import torch
+    B, N, d, dt = _dims(x, n_g)
+    m, n = _coef(a, b, n_g)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    dA = torch.empty((n_g, m + 1), dtype=torch.float32, device=x.device)
+    dB = torch.empty((n_g, n), dtype=torch.float32, device=x.device)
+    wsb = grkan_backward_workspace_bytes(B, N, d, n_g, m, n, dt)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=x.device)
+    _check(grkan_forward_backward(x, dy, a, b, y, dx, dA, dB, B, N, d, n_g, m, n, dt, ws,
+                                  ws.numel(), flags, stream), "grkan_forward_backward")
+    return y, dx, dA, dB

@@ -6,6 +6,8 @@ Bytes (element size es = 4 for float32 I/O, 2 for bf16):
   backward  read x and dy, write dx           3 es   (stage 1; the partials,
             coefficients and the merge add < 1 MB per call and are left out)
   step      forward + backward                5 es
+  forward_backward  read x and dy, write y and dx   4 es   (the recompute
+            variant: one pass over x and dy for both outputs)
 Floating point: the forward's extra operations per input are 2m + 2n + 3
 ("FlashKAT: Understanding and Addressing Performance Bottlenecks in the
 Kolmogorov-Arnold Transformer", paper notes, section "Insight 2": the GR-KAN
@@ -20,7 +22,8 @@ def element_size(dtype):
 
 def bytes_per_element(phase, dtype):
     es = element_size(dtype)
-    return {"forward": 2 * es, "backward": 3 * es, "step": 5 * es}[phase]
+    return {"forward": 2 * es, "backward": 3 * es, "step": 5 * es,
+            "forward_backward": 4 * es}[phase]
 
 
 def forward_flops_per_element(m, n):

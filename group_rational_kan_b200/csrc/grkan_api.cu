@@ -283,7 +283,7 @@ grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float
   return cuda_status(e, "forward (TMA) launch");
 }
 
-grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx,
+grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx, void* y,
                               const float* a, const float* b, float* ws, long long ws_T,
                               long long tile0, cudaStream_t st) {
   CUtensorMap mx, mdy;
@@ -291,7 +291,7 @@ grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void
   grk::TmaGeom geom = make_geom(p, p.bbox);
   geom.ws_T = ws_T;
   geom.ws_tile0 = tile0;
-  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, dx, a, b, ws,
+  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, dx, y, a, b, ws,
                                       sm_count(), st);
   return cuda_status(e, "backward (TMA) launch");
 }
@@ -324,12 +324,22 @@ grkan_status_t do_forward(const void* x, void* y, const float* a, const float* b
 
 // Stage 1 into the workspace; the partials of this call's tiles go to tiles
 // [tile0, tile0 + p.T) of a workspace laid out for ws_T tiles (a whole tensor).
+// Stage 1 into the workspace; the partials of this call's tiles go to tiles
+// [tile0, tile0 + p.T) of a workspace laid out for ws_T tiles (a whole tensor).
+// With y != nullptr the forward output is written too (one pass over x, dy on the
+// TMA path; a forward kernel first on the generic path).
 grkan_status_t do_partials_at(const Plan& p, const void* x, const void* dy, const float* a,
-                              const float* b, void* dx, void* ws, long long ws_T, long long tile0,
-                              uint32_t flags, cudaStream_t st) {
+                              const float* b, void* dx, void* y, void* ws, long long ws_T,
+                              long long tile0, uint32_t flags, cudaStream_t st) {
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
-  if (choose_bwd_path(p, x, dy, dx, flags) == 1)
-    return launch_tma_bwd(p, x, dy, dx, a, b, (float*)ws, ws_T, tile0, st);
+  if (choose_bwd_path(p, x, dy, dx, flags) == 1 && (!y || aligned16(y)))
+    return launch_tma_bwd(p, x, dy, dx, y, a, b, (float*)ws, ws_T, tile0, st);
+  if (y) {
+    cudaError_t e = (p.dtype == GRKAN_F32) ? launch_generic_fwd<grk::IoF32>(p, x, y, a, b, st)
+                                           : launch_generic_fwd<grk::IoBF16>(p, x, y, a, b, st);
+    grkan_status_t s = cuda_status(e, "forward (generic) launch");
+    if (s != GRKAN_OK) return s;
+  }
   cudaError_t e =
       (p.dtype == GRKAN_F32)
           ? launch_generic_bwd<grk::IoF32>(p, x, dy, dx, a, b, (float*)ws, ws_T, tile0, st)
@@ -349,7 +359,7 @@ grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const f
   if (overlaps(ws, p.ws_bytes, x, bytes) || overlaps(ws, p.ws_bytes, dy, bytes) ||
       overlaps(ws, p.ws_bytes, dx, bytes))
     return GRKAN_ERR_ALIAS;
-  return do_partials_at(p, x, dy, a, b, dx, ws, p.T, 0, flags, st);
+  return do_partials_at(p, x, dy, a, b, dx, nullptr, ws, p.T, 0, flags, st);
 }
 
 grkan_status_t do_merge(const Plan& p, const void* ws, size_t ws_bytes, float* dA, float* dB,
@@ -575,6 +585,35 @@ grkan_status_t grkan_backward_noalloc(const void* x, const void* dy, const float
   return do_merge(p, ws, GRKAN_NOALLOC_WORKSPACE_BYTES, dA, dB, nullptr, st);
 }
 
+grkan_status_t grkan_forward_backward(const void* x, const void* dy, const float* a,
+                                      const float* b, void* y, void* dx, float* dA, float* dB,
+                                      int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
+                                      int32_t n, grkan_dtype_t dtype, void* workspace,
+                                      size_t workspace_bytes, uint32_t flags, void* stream) {
+  if (flags & ~GRKAN_FLAG_GENERIC) return GRKAN_ERR_FLAGS;
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (!dA || (p.n > 0 && !dB)) return GRKAN_ERR_NULL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.T > 0) {
+    if (!x || !dy || !dx || !y) return GRKAN_ERR_NULL;
+    if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+    if (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace))
+      return GRKAN_ERR_WORKSPACE;
+    const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
+    if (bad_alias(x, dx, bytes) || bad_alias(dy, dx, bytes) || overlaps(y, bytes, x, bytes) ||
+        overlaps(y, bytes, dy, bytes) || overlaps(y, bytes, dx, bytes))
+      return GRKAN_ERR_ALIAS;
+    if (overlaps(workspace, p.ws_bytes, x, bytes) || overlaps(workspace, p.ws_bytes, dy, bytes) ||
+        overlaps(workspace, p.ws_bytes, dx, bytes) || overlaps(workspace, p.ws_bytes, y, bytes))
+      return GRKAN_ERR_ALIAS;
+    s = do_partials_at(p, x, dy, a, b, dx, y, workspace, p.T, 0, flags, st);
+    if (s != GRKAN_OK) return s;
+  }
+  return do_merge(p, workspace, workspace_bytes, dA, dB, nullptr, st);
+}
+
 size_t grkan_step_host_scratch_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
                                      int32_t n, grkan_dtype_t dtype, int64_t chunk_rows) {
   Plan p;
@@ -659,7 +698,7 @@ grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const fl
         s = cuda_status(e, "forward (generic) launch");
       }
       if (s != GRKAN_OK) return s;
-      s = do_partials_at(pc, sx, sdy, a, b, sdx, ws, p.T, r0 / p.S, 0u, hp->s_comp);
+      s = do_partials_at(pc, sx, sdy, a, b, sdx, nullptr, ws, p.T, r0 / p.S, 0u, hp->s_comp);
       if (s != GRKAN_OK) return s;
       GRK_TRY(cudaEventRecord(hp->comp[slot], hp->s_comp), "cudaEventRecord");
       // outputs out

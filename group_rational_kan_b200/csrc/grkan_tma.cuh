@@ -251,7 +251,8 @@ struct Acc54 {
 };
 
 // dx for a pair of elements; adds t x^i and -t y s x^j to the sums.
-__device__ __forceinline__ float2 bwd_pair(const Coef54& c, float2 x, float2 dy, Acc54& acc) {
+__device__ __forceinline__ float2 bwd_pair(const Coef54& c, float2 x, float2 dy, Acc54& acc,
+                                           float2* y_out = nullptr) {
   const float2 x2 = mul2(x, x);
   const float2 x3 = mul2(x2, x);
   const float2 x4 = mul2(x2, x2);
@@ -265,6 +266,7 @@ __device__ __forceinline__ float2 bwd_pair(const Coef54& c, float2 x, float2 dy,
   const float2 dQ = fma2(x2, fma2(c.jb4, x, c.jb3), fma2(c.jb2, x, c.b1));
   const float2 r = make_float2(rcp_approx(1.f + fabsf(Q.x)), rcp_approx(1.f + fabsf(Q.y)));
   const float2 y = mul2(P, r);
+  if (y_out) *y_out = y;
   const float2 t = mul2(dy, r);
   const float2 nu = mul2(t, make_float2(neg_y_sign(y.x, Q.x), neg_y_sign(y.y, Q.y)));
   acc.a0 = add2(acc.a0, t);
@@ -538,10 +540,13 @@ __device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile)
   return (int)((left + g.SCw - 1) / g.SCw);
 }
 
-template <class IO>
+// kWithY: also write y (the forward output recomputed on the way), for
+// training that recomputes the activation during the backward pass.
+template <class IO, bool kWithY>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
-        typename IO::T* __restrict__ dx, const float* __restrict__ a,
+        typename IO::T* __restrict__ dx, typename IO::T* __restrict__ yout,
+        const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
   using S_ = Shape<IO>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -629,6 +634,9 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         const uint4* gb = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot);
         const int r0 = rb * geom.SCw;  // row of the box within the tile
         typename IO::T* dxo = dxt + (long long)r0 * geom.d + bx * geom.bw;
+        typename IO::T* yo = nullptr;
+        if constexpr (kWithY)
+          yo = yout + (tile * geom.S + r0) * geom.d + g * geom.dg + bx * geom.bw;
 #pragma unroll
         for (int h = 0; h < S_::kBwdHalves; ++h) {
           uint4 xv[kBwdVec], gv[kBwdVec];
@@ -663,23 +671,39 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
             const int sl = h * kBwdVec + it;
             // rows past the end arrive zero-filled from TMA: they add exact
             // zeros to the sums and are not stored
-            uint4 o;
+            uint4 o, oy;
+            float2 y0, y1, y2, y3;
             if constexpr (IO::kBytes == 2) {
-              o.x = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc));
-              o.y = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc));
-              o.z = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc));
-              o.w = f2_to_bf16x2(bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc));
+              o.x = f2_to_bf16x2(
+                  bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc, kWithY ? &y0 : nullptr));
+              o.y = f2_to_bf16x2(
+                  bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc, kWithY ? &y1 : nullptr));
+              o.z = f2_to_bf16x2(
+                  bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc, kWithY ? &y2 : nullptr));
+              o.w = f2_to_bf16x2(
+                  bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc, kWithY ? &y3 : nullptr));
+              if constexpr (kWithY)
+                oy = make_uint4(f2_to_bf16x2(y0), f2_to_bf16x2(y1), f2_to_bf16x2(y2),
+                                f2_to_bf16x2(y3));
             } else {
               const float2 p0 = bwd_pair(
                   c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
-                  make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc);
+                  make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc,
+                  kWithY ? &y0 : nullptr);
               const float2 p1 = bwd_pair(
                   c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
-                  make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc);
+                  make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc,
+                  kWithY ? &y1 : nullptr);
               o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
                              __float_as_uint(p1.y));
+              if constexpr (kWithY)
+                oy = make_uint4(__float_as_uint(y0.x), __float_as_uint(y0.y),
+                                __float_as_uint(y1.x), __float_as_uint(y1.y));
             }
-            if (r0 + lm.row[sl] < rows_left) store16(dxo + lm.off[sl], o);
+            if (r0 + lm.row[sl] < rows_left) {
+              store16(dxo + lm.off[sl], o);
+              if constexpr (kWithY) store16(yo + lm.off[sl], oy);
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -721,15 +745,16 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 // largest shared-memory carveout. One cache per kernel instantiation (the
 // instantiations share a function-pointer type, so the cache is keyed on the
 // template arguments); set once per device.
-template <class IO, bool kBackward>
+template <class IO, int kKernel>  // 0 forward, 1 backward, 2 backward with y
 inline cudaError_t ensure_smem(unsigned bytes) {
   static int done_for_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (done_for_device == dev) return cudaSuccess;
-  const void* fn = kBackward ? reinterpret_cast<const void*>(bwd_tma<IO>)
-                             : reinterpret_cast<const void*>(fwd_tma<IO>);
+  const void* fn = kKernel == 1   ? reinterpret_cast<const void*>(bwd_tma<IO, false>)
+                   : kKernel == 2 ? reinterpret_cast<const void*>(bwd_tma<IO, true>)
+                                  : reinterpret_cast<const void*>(fwd_tma<IO>);
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -757,36 +782,41 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   cudaError_t e;
   if (bf16) {
     const unsigned smem = fwd_smem_bytes<IoBF16>();
-    if ((e = ensure_smem<IoBF16, false>(smem)) != cudaSuccess) return e;
+    if ((e = ensure_smem<IoBF16, 0>(smem)) != cudaSuccess) return e;
     fwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoBF16::T*)y, a, b, g);
   } else {
     const unsigned smem = fwd_smem_bytes<IoF32>();
-    if ((e = ensure_smem<IoF32, false>(smem)) != cudaSuccess) return e;
+    if ((e = ensure_smem<IoF32, 0>(smem)) != cudaSuccess) return e;
     fwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoF32::T*)y, a, b, g);
   }
   return cudaGetLastError();
 }
 
+template <class IO, bool kWithY>
+inline cudaError_t launch_bwd_tma_t(const TmaGeom& g, const CUtensorMap& mx,
+                                    const CUtensorMap& mdy, void* dx, void* y, const float* a,
+                                    const float* b, float* ws, long long grid, cudaStream_t st) {
+  const unsigned smem = bwd_smem_bytes<IO>();
+  cudaError_t e = ensure_smem<IO, kWithY ? 2 : 1>(smem);
+  if (e != cudaSuccess) return e;
+  bwd_tma<IO, kWithY><<<(unsigned)grid, kThreads, smem, st>>>(
+      mx, mdy, (typename IO::T*)dx, (typename IO::T*)y, a, b, ws, g);
+  return cudaGetLastError();
+}
+
+// y == nullptr: backward only; otherwise also write the recomputed forward y.
 inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
-                                  const CUtensorMap& mdy, void* dx, const float* a,
+                                  const CUtensorMap& mdy, void* dx, void* y, const float* a,
                                   const float* b, float* ws, int sms, cudaStream_t st) {
   if (g.box_bytes > bwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long units = g.T * g.n_g;
   long long grid = sms;
   if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
-  cudaError_t e;
-  if (bf16) {
-    const unsigned smem = bwd_smem_bytes<IoBF16>();
-    if ((e = ensure_smem<IoBF16, true>(smem)) != cudaSuccess) return e;
-    bwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, mdy, (IoBF16::T*)dx, a, b,
-                                                                ws, g);
-  } else {
-    const unsigned smem = bwd_smem_bytes<IoF32>();
-    if ((e = ensure_smem<IoF32, true>(smem)) != cudaSuccess) return e;
-    bwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, mdy, (IoF32::T*)dx, a, b, ws,
-                                                               g);
-  }
-  return cudaGetLastError();
+  if (bf16)
+    return y ? launch_bwd_tma_t<IoBF16, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+             : launch_bwd_tma_t<IoBF16, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+  return y ? launch_bwd_tma_t<IoF32, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+           : launch_bwd_tma_t<IoF32, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
 }
 
 inline cudaError_t read_device_error(uint32_t* out, cudaStream_t st) {

@@ -116,6 +116,20 @@ GRKAN_API grkan_status_t grkan_backward_ex(const void* x, const void* dy, const 
                                  void* workspace, size_t workspace_bytes, uint32_t flags,
                                  void* stream);
 
+/* Forward and backward fused in one pass over x and dy, for training that
+ * recomputes the activation in the backward pass (activation checkpointing):
+ * writes y (as grkan_forward) and dx, dA, dB (as grkan_backward). Reads x and dy
+ * once and writes y and dx once: 4 element sizes of traffic per element instead
+ * of 5 for the two separate calls. y may not overlap x, dy or dx; dx may equal
+ * dy. flags: 0 or GRKAN_FLAG_GENERIC. */
+GRKAN_API grkan_status_t grkan_forward_backward(const void* x, const void* dy, const float* a,
+                                                const float* b, void* y, void* dx, float* dA,
+                                                float* dB, int64_t B, int64_t N, int64_t d,
+                                                int32_t n_g, int32_t m, int32_t n,
+                                                grkan_dtype_t dtype, void* workspace,
+                                                size_t workspace_bytes, uint32_t flags,
+                                                void* stream);
+
 /* Stage 1 alone: dx, plus one float32 partial sum per (row tile, group,
  * coefficient) into the workspace. */
 GRKAN_API grkan_status_t grkan_backward_partials(const void* x, const void* dy, const float* a,

@@ -224,3 +224,36 @@ def test_partials_merge_and_sums64():
     ref = grk.backward(tx, tdy, ta, tb, w.n_g)
     assert torch.equal(dx, ref[0]) and torch.equal(dA, ref[1]) and torch.equal(dB, ref[2])
     assert torch.equal(s64[:, :6].float(), dA) and torch.equal(s64[:, 6:].float(), dB)
+
+
+@pytest.mark.parametrize("flags", [0, grk.FLAG_GENERIC], ids=["auto", "generic"])
+@pytest.mark.parametrize("name", ["tiny", "kat_t_ragged", "kat_b_ragged", "stress_ng64",
+                                  "one_row_bf16", "odd_f32_dg10", "deg_3_2"])
+def test_fused_recompute_parity(name, flags):
+    """grkan_forward_backward (y recomputed inside the backward pass): y against
+    the oracle, and dx, dA, dB the same bits as the separate backward call."""
+    w, x, dy, a, b, y_ref, ky, dx_ref, ex, g_ref = case_data(name)
+    tx, tdy, ta, tb = _dev(w, x, dy, a, b)
+    y, dx, dA, dB = grk.forward_backward(tx, tdy, ta, tb, w.n_g, flags=flags)
+    sdx, sdA, sdB = grk.backward(tx, tdy, ta, tb, w.n_g, flags=flags)
+    torch.cuda.synchronize()
+    rtol = RTOL[w.dtype]
+    check_y(to_f64(y), y_ref, ky, rtol, "%s fused y" % name)
+    check_dx(to_f64(dx), dx_ref, ex, rtol, "%s fused dx" % name)
+    check_coef(dA.cpu().numpy(), dB.cpu().numpy(), g_ref, what=name)
+    assert torch.equal(dx, sdx) and torch.equal(dA, sdA) and torch.equal(dB, sdB)
+    assert grk.grkan_device_error()[1] == 0
+
+
+def test_fused_recompute_rejects_overlapping_y():
+    w, x, dy, a, b = case_data("kat_t_ragged")[:5]
+    tx, tdy, ta, tb = _dev(w, x, dy, a, b)
+    dx = torch.empty_like(tx)
+    dA = torch.empty(w.n_g, w.m + 1, device="cuda")
+    dB = torch.empty(w.n_g, w.n, device="cuda")
+    wsb = grk.grkan_backward_workspace_bytes(w.rows, 1, w.d, w.n_g, w.m, w.n, w.dtype)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    for y in (tx, tdy, dx):
+        st = grk.grkan_forward_backward(tx, tdy, ta, tb, y, dx, dA, dB, w.rows, 1, w.d, w.n_g,
+                                        w.m, w.n, w.dtype, ws, wsb)
+        assert st == 7  # GRKAN_ERR_ALIAS
