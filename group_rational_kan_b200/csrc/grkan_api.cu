@@ -259,6 +259,9 @@ grk::TmaGeom make_geom(const Plan& p, const Box& bx) {
   g.box_bytes = bx.bytes;
   g.m = p.m;
   g.n = p.n;
+  g.nrb_full = (int)((p.S + bx.scw - 1) / bx.scw);
+  const long long last = p.T > 0 ? p.rows - (p.T - 1) * p.S : 0;
+  g.nrb_last = (int)((last + bx.scw - 1) / bx.scw);
   return g;
 }
 

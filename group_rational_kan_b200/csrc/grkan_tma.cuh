@@ -44,6 +44,8 @@ struct TmaGeom {
   int nbox;             // boxes per group row = dg / bw
   unsigned box_bytes;   // SCw * bw * element size
   int m, n;             // degrees
+  int nrb_full;         // row blocks (boxes of SCw rows) of a full tile: ceil(S / SCw)
+  int nrb_last;         // row blocks of the last tile
 };
 
 // Launch shape (compile-time; the defaults are the tuned configuration).
@@ -82,7 +84,10 @@ struct TmaGeom {
 
 constexpr int kWarps = GRK_WARPS;
 constexpr int kThreads = kWarps * 32;
-constexpr int kBwdVec = 3;  // 16-byte vectors per lane and tensor in one backward pass
+#ifndef GRK_BWD_VEC
+#define GRK_BWD_VEC 3
+#endif
+constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor in one backward pass
 
 template <class IO>
 struct Shape;
@@ -533,28 +538,69 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
 // (tile, g), coefficient k goes to ws[(g * 10 + k) * ws_T + ws_tile0 + tile].
 
 
-// Row blocks of tile `tile`: ceil(min(S, rows - tile * S) / SCw).
+// Row blocks of tile `tile`: ceil(min(S, rows - tile * S) / SCw); only the last
+// tile can be short.
 __device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile) {
-  long long left = g.rows - tile * g.S;
-  if (left > g.S) left = g.S;
-  return (int)((left + g.SCw - 1) / g.SCw);
+  return tile == g.T - 1 ? g.nrb_last : g.nrb_full;
+}
+
+// Coefficients of every group in the CTA's shared memory after the warps'
+// regions, 20 floats per group (a_0..a_5, i a_i for i = 2..5, b_1..b_4, j b_j for
+// j = 2..4, padding), used when n_g <= kTableGroups; larger group counts stage
+// one group at a time in the warp's own slot. Scalars, not pairs: a pair built
+// in registers from one scalar lets the compiler keep one register per
+// coefficient.
+constexpr int kTableGroups = 64;
+constexpr int kTabFloats = 20;
+__host__ __device__ constexpr unsigned coef_table_bytes() {
+  return (unsigned)(kTableGroups * kTabFloats * 4);
+}
+
+__device__ __forceinline__ void build_coef_table(float* tab, const float* a, const float* b,
+                                                 int n_g) {
+  for (int e = threadIdx.x; e < n_g * kTabFloats; e += blockDim.x) {
+    const int g = e / kTabFloats;
+    const int k = e - g * kTabFloats;
+    float v = 0.f;
+    if (k < 6) v = __ldg(a + g * 6 + k);                                  // a_0..a_5
+    else if (k < 10) v = (float)(k - 4) * __ldg(a + g * 6 + (k - 4));    // i a_i, i = 2..5
+    else if (k < 14) v = __ldg(b + g * 4 + (k - 10));                    // b_1..b_4
+    else if (k < 17) v = (float)(k - 12) * __ldg(b + g * 4 + (k - 13));  // j b_j, j = 2..4
+    tab[e] = v;
+  }
+}
+
+__device__ __forceinline__ void load_coef(const float* t, Coef54& c) {
+  const float4* q = reinterpret_cast<const float4*>(t);
+  const float4 v0 = q[0], v1 = q[1], v2 = q[2], v3 = q[3], v4 = q[4];
+  c.a0 = f2(v0.x); c.a1 = f2(v0.y); c.a2 = f2(v0.z); c.a3 = f2(v0.w);
+  c.a4 = f2(v1.x); c.a5 = f2(v1.y); c.ia2 = f2(v1.z); c.ia3 = f2(v1.w);
+  c.ia4 = f2(v2.x); c.ia5 = f2(v2.y); c.b1 = f2(v2.z); c.b2 = f2(v2.w);
+  c.b3 = f2(v3.x); c.b4 = f2(v3.y); c.jb2 = f2(v3.z); c.jb3 = f2(v3.w);
+  c.jb4 = f2(v4.x);
 }
 
 // kWithY: also write y (the forward output recomputed on the way), for
 // training that recomputes the activation during the backward pass.
-template <class IO, bool kWithY>
+// kFull: every 16-byte vector slot of a lane holds box data (the box is exactly
+// 32 * NV vectors), so the loads need no guard.
+template <class IO, bool kWithY, bool kFull>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
         typename IO::T* __restrict__ dx, typename IO::T* __restrict__ yout,
         const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
   using S_ = Shape<IO>;
+  using T = typename IO::T;
+  constexpr int NV = kBwdVec * S_::kBwdHalves;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const WarpLayout L(geom.box_bytes, 2, S_::kBwdStages);
   unsigned char* base = smem + warp * L.per_warp;
   float* cslot = reinterpret_cast<float*>(base + L.coef_off);
+  float* ctab = reinterpret_cast<float*>(smem + kWarps * L.per_warp);
+  const bool use_tab = geom.n_g <= kTableGroups;
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * S_::kBwdStages;
   const long long gw = (long long)blockIdx.x * kWarps + warp;
@@ -572,7 +618,8 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
       prefetch_map(&mdy);
     }
   }
-  __syncwarp();
+  if (use_tab) build_coef_table(ctab, a, b, geom.n_g);
+  __syncthreads();
 
   // issue cursor (lane 0): unit (tile, g) = iu.hi, iu.lo; box (irb, ibx) of inrb row blocks
   Cursor3 iu;
@@ -601,8 +648,13 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     for (int s = 0; s < S_::kBwdStages && iu.hi < geom.T; ++s) issue();
   __syncwarp();
 
-  LaneMap<IO, kBwdVec * S_::kBwdHalves> lm;
+  // per-lane byte offsets of the lane's vectors from a box's origin in global memory
+  LaneMap<IO, NV> lm;
   lm.init(geom, lane, geom.d);
+  int boff[NV];
+#pragma unroll
+  for (int sl = 0; sl < NV; ++sl) boff[sl] = lm.off[sl] * (int)sizeof(T);
+  const long long row_bytes = geom.d * (long long)sizeof(T);
   Coef54 c;
   int cur_g = -1;
   Acc54 acc;
@@ -615,13 +667,19 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     const int g = cu.lo;
     const int nrb = tile_row_blocks(geom, tile);
     if (g != cur_g) {
-      stage_coefficients(cslot, a, b, g, lane, c);
+      if (use_tab) load_coef(ctab + g * kTabFloats, c);
+      else stage_coefficients(cslot, a, b, g, lane, c);
       cur_g = g;
     }
     acc.zero();
-    typename IO::T* dxt = dx + tile * geom.S * geom.d + g * geom.dg;
-    const long long rows_left = geom.rows - tile * geom.S;
+    const long long left = geom.rows - tile * geom.S;
+    const int rows_left = left < geom.S ? (int)left : (int)geom.S;
+    const long long tile_off = (tile * geom.S * geom.d + (long long)g * geom.dg) * sizeof(T);
+    char* dxt = reinterpret_cast<char*>(dx) + tile_off;
+    char* yt = kWithY ? reinterpret_cast<char*>(yout) + tile_off : nullptr;
     for (int rb = 0; rb < nrb && ok; ++rb) {
+      const int r0 = rb * geom.SCw;     // row of the box within the tile
+      const int lim = rows_left - r0;   // lane vectors in rows >= lim are past the end
       for (int bx = 0; bx < geom.nbox; ++bx, ++q) {
         const int s = q % S_::kBwdStages;
         const uint32_t ph = (uint32_t)(q / S_::kBwdStages) & 1;
@@ -630,22 +688,20 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
           ok = false;
           break;
         }
-        const uint4* xb = reinterpret_cast<const uint4*>(base + s * L.stage);
-        const uint4* gb = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot);
-        const int r0 = rb * geom.SCw;  // row of the box within the tile
-        typename IO::T* dxo = dxt + (long long)r0 * geom.d + bx * geom.bw;
-        typename IO::T* yo = nullptr;
-        if constexpr (kWithY)
-          yo = yout + (tile * geom.S + r0) * geom.d + g * geom.dg + bx * geom.bw;
+        const uint4* xl = reinterpret_cast<const uint4*>(base + s * L.stage) + lane;
+        const uint4* gl = reinterpret_cast<const uint4*>(base + s * L.stage + L.box_slot) + lane;
+        const long long box_off = (long long)r0 * row_bytes + (long long)bx * geom.bw * sizeof(T);
+        char* dxo = dxt + box_off;
+        char* yo = kWithY ? yt + box_off : nullptr;
 #pragma unroll
         for (int h = 0; h < S_::kBwdHalves; ++h) {
           uint4 xv[kBwdVec], gv[kBwdVec];
 #pragma unroll
           for (int it = 0; it < kBwdVec; ++it) {
             const int sl = h * kBwdVec + it;
-            if (lm.row[sl] < geom.SCw) {
-              xv[it] = xb[lane + 32 * sl];
-              gv[it] = gb[lane + 32 * sl];
+            if (kFull || lm.row[sl] < geom.SCw) {
+              xv[it] = xl[32 * sl];
+              gv[it] = gl[32 * sl];
             } else {
               xv[it] = make_uint4(0, 0, 0, 0);
               gv[it] = make_uint4(0, 0, 0, 0);
@@ -700,9 +756,9 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
                 oy = make_uint4(__float_as_uint(y0.x), __float_as_uint(y0.y),
                                 __float_as_uint(y1.x), __float_as_uint(y1.y));
             }
-            if (r0 + lm.row[sl] < rows_left) {
-              store16(dxo + lm.off[sl], o);
-              if constexpr (kWithY) store16(yo + lm.off[sl], oy);
+            if (lm.row[sl] < lim) {
+              store16(dxo + boff[sl], o);
+              if constexpr (kWithY) store16(yo + boff[sl], oy);
             }
           }
         }
@@ -742,19 +798,16 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 // --- host-side launchers ---------------------------------------------------------
 
 // Raise a kernel's dynamic shared-memory limit to what it uses and ask for the
-// largest shared-memory carveout. One cache per kernel instantiation (the
-// instantiations share a function-pointer type, so the cache is keyed on the
-// template arguments); set once per device.
-template <class IO, int kKernel>  // 0 forward, 1 backward, 2 backward with y
+// largest shared-memory carveout; once per kernel and device (the cache is keyed
+// on the kernel itself).
+template <auto Kernel>
 inline cudaError_t ensure_smem(unsigned bytes) {
   static int done_for_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (done_for_device == dev) return cudaSuccess;
-  const void* fn = kKernel == 1   ? reinterpret_cast<const void*>(bwd_tma<IO, false>)
-                   : kKernel == 2 ? reinterpret_cast<const void*>(bwd_tma<IO, true>)
-                                  : reinterpret_cast<const void*>(fwd_tma<IO>);
+  const void* fn = reinterpret_cast<const void*>(Kernel);
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -770,7 +823,8 @@ inline unsigned fwd_smem_bytes() {
 }
 template <class IO>
 inline unsigned bwd_smem_bytes() {
-  return kWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp;
+  return kWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp +
+         coef_table_bytes();
 }
 
 inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx, void* y,
@@ -782,26 +836,39 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   cudaError_t e;
   if (bf16) {
     const unsigned smem = fwd_smem_bytes<IoBF16>();
-    if ((e = ensure_smem<IoBF16, 0>(smem)) != cudaSuccess) return e;
+    if ((e = ensure_smem<fwd_tma<IoBF16>>(smem)) != cudaSuccess) return e;
     fwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoBF16::T*)y, a, b, g);
   } else {
     const unsigned smem = fwd_smem_bytes<IoF32>();
-    if ((e = ensure_smem<IoF32, 0>(smem)) != cudaSuccess) return e;
+    if ((e = ensure_smem<fwd_tma<IoF32>>(smem)) != cudaSuccess) return e;
     fwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoF32::T*)y, a, b, g);
   }
   return cudaGetLastError();
 }
 
-template <class IO, bool kWithY>
+template <class IO, bool kWithY, bool kFull>
 inline cudaError_t launch_bwd_tma_t(const TmaGeom& g, const CUtensorMap& mx,
                                     const CUtensorMap& mdy, void* dx, void* y, const float* a,
                                     const float* b, float* ws, long long grid, cudaStream_t st) {
   const unsigned smem = bwd_smem_bytes<IO>();
-  cudaError_t e = ensure_smem<IO, kWithY ? 2 : 1>(smem);
+  cudaError_t e = ensure_smem<bwd_tma<IO, kWithY, kFull>>(smem);
   if (e != cudaSuccess) return e;
-  bwd_tma<IO, kWithY><<<(unsigned)grid, kThreads, smem, st>>>(
+  bwd_tma<IO, kWithY, kFull><<<(unsigned)grid, kThreads, smem, st>>>(
       mx, mdy, (typename IO::T*)dx, (typename IO::T*)y, a, b, ws, g);
   return cudaGetLastError();
+}
+
+template <class IO>
+inline cudaError_t launch_bwd_tma_io(const TmaGeom& g, const CUtensorMap& mx,
+                                     const CUtensorMap& mdy, void* dx, void* y, const float* a,
+                                     const float* b, float* ws, long long grid, cudaStream_t st) {
+  // every lane vector slot used: the box is exactly 32 lanes x NV vectors
+  const bool full = g.box_bytes == 16u * 32u * (unsigned)(kBwdVec * Shape<IO>::kBwdHalves);
+  if (full)
+    return y ? launch_bwd_tma_t<IO, true, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+             : launch_bwd_tma_t<IO, false, true>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+  return y ? launch_bwd_tma_t<IO, true, false>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+           : launch_bwd_tma_t<IO, false, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
 }
 
 // y == nullptr: backward only; otherwise also write the recomputed forward y.
@@ -812,11 +879,8 @@ inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   const long long units = g.T * g.n_g;
   long long grid = sms;
   if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
-  if (bf16)
-    return y ? launch_bwd_tma_t<IoBF16, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-             : launch_bwd_tma_t<IoBF16, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
-  return y ? launch_bwd_tma_t<IoF32, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-           : launch_bwd_tma_t<IoF32, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+  return bf16 ? launch_bwd_tma_io<IoBF16>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+              : launch_bwd_tma_io<IoF32>(g, mx, mdy, dx, y, a, b, ws, grid, st);
 }
 
 inline cudaError_t read_device_error(uint32_t* out, cudaStream_t st) {
