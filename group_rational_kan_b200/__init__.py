@@ -18,6 +18,7 @@ __all__ = [
     "grkan_backward_partials", "grkan_backward_merge", "grkan_backward_workspace_bytes",
     "grkan_merge_ranks", "grkan_backward_noalloc", "NOALLOC_WORKSPACE_BYTES",
     "grkan_step_host", "grkan_step_host_scratch_bytes", "grkan_forward_backward",
+    "grkan_backward_atomic", "ATOMIC_PER_ELEMENT", "ATOMIC_PER_BLOCK",
     "forward_backward",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
     "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
@@ -66,6 +67,8 @@ def _load():
         "grkan_backward_merge": (S, [P, SZ, P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int,
                                      P]),
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
+        "grkan_backward_atomic": (S, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
+                                      ctypes.c_int, I32, I32, P]),
         "grkan_forward_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                        ctypes.c_int, P, SZ, U32, P]),
         "grkan_step_host_scratch_bytes": (SZ, [I64, I64, I64, I32, I32, I32, ctypes.c_int, I64]),
@@ -171,6 +174,17 @@ def grkan_backward_noalloc(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, s
     callers that cannot allocate device memory per call)."""
     return lib().grkan_backward_noalloc(_ptr(x), _ptr(dy), _ptr(a), _ptr(b), _ptr(dx), _ptr(dA),
                                         _ptr(dB), B, N, d, n_g, m, n, dtype, _stream(stream))
+
+
+ATOMIC_PER_ELEMENT = 1
+ATOMIC_PER_BLOCK = 2
+
+
+def grkan_backward_atomic(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, mode, block_rows=0,
+                          stream=None):
+    return lib().grkan_backward_atomic(_ptr(x), _ptr(dy), _ptr(a), _ptr(b), _ptr(dx), _ptr(dA),
+                                       _ptr(dB), B, N, d, n_g, m, n, dtype, mode, block_rows,
+                                       _stream(stream))
 
 
 def grkan_forward_backward(x, dy, a, b, y, dx, dA, dB, B, N, d, n_g, m, n, dtype, workspace,

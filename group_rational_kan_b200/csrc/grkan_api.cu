@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "grkan.h"
+#include "grkan_atomic.cuh"
 #include "grkan_common.cuh"
 #include "grkan_generic.cuh"
 #include "grkan_merge.cuh"
@@ -327,8 +328,6 @@ grkan_status_t do_forward(const void* x, void* y, const float* a, const float* b
 
 // Stage 1 into the workspace; the partials of this call's tiles go to tiles
 // [tile0, tile0 + p.T) of a workspace laid out for ws_T tiles (a whole tensor).
-// Stage 1 into the workspace; the partials of this call's tiles go to tiles
-// [tile0, tile0 + p.T) of a workspace laid out for ws_T tiles (a whole tensor).
 // With y != nullptr the forward output is written too (one pass over x, dy on the
 // TMA path; a forward kernel first on the generic path).
 grkan_status_t do_partials_at(const Plan& p, const void* x, const void* dy, const float* a,
@@ -548,6 +547,62 @@ grkan_status_t grkan_backward(const void* x, const void* dy, const float* a, con
                               void* workspace, size_t workspace_bytes, void* stream) {
   return grkan_backward_ex(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, workspace,
                            workspace_bytes, 0u, stream);
+}
+
+grkan_status_t grkan_backward_atomic(const void* x, const void* dy, const float* a,
+                                     const float* b, void* dx, float* dA, float* dB, int64_t B,
+                                     int64_t N, int64_t d, int32_t n_g, int32_t m, int32_t n,
+                                     grkan_dtype_t dtype, int32_t mode, int32_t block_rows,
+                                     void* stream) {
+  if (mode != GRKAN_ATOMIC_PER_ELEMENT && mode != GRKAN_ATOMIC_PER_BLOCK) return GRKAN_ERR_FLAGS;
+  if (block_rows < 0) return GRKAN_ERR_SHAPE;
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (!dA || (p.n > 0 && !dB)) return GRKAN_ERR_NULL;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(dA, 0, sizeof(float) * p.n_g * (p.m + 1), st);
+  if (e == cudaSuccess && p.n > 0) e = cudaMemsetAsync(dB, 0, sizeof(float) * p.n_g * p.n, st);
+  if ((s = cuda_status(e, "grkan_backward_atomic zeroing")) != GRKAN_OK) return s;
+  if (p.T == 0) return GRKAN_OK;
+  if (!x || !dy || !dx) return GRKAN_ERR_NULL;
+  if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+  const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
+  if (bad_alias(x, dx, bytes) || bad_alias(dy, dx, bytes)) return GRKAN_ERR_ALIAS;
+  const bool f32 = p.dtype == GRKAN_F32;
+  if (mode == GRKAN_ATOMIC_PER_ELEMENT) {
+    const long long elems = p.rows * p.d;
+    long long blocks = (elems + grk::kAtomicThreads - 1) / grk::kAtomicThreads;
+    const long long cap = (long long)sm_count() * 32;
+    if (blocks > cap) blocks = cap;
+    if (f32)
+      grk::bwd_atomic_element<grk::IoF32, GRKAN_MAX_M, GRKAN_MAX_N>
+          <<<(unsigned)blocks, grk::kAtomicThreads, 0, st>>>(
+              (const float*)x, (const float*)dy, (float*)dx, a, b, dA, dB, elems, p.d,
+              (int)p.dg, p.m, p.n);
+    else
+      grk::bwd_atomic_element<grk::IoBF16, GRKAN_MAX_M, GRKAN_MAX_N>
+          <<<(unsigned)blocks, grk::kAtomicThreads, 0, st>>>(
+              (const grk::IoBF16::T*)x, (const grk::IoBF16::T*)dy, (grk::IoBF16::T*)dx, a, b,
+              dA, dB, elems, p.d, (int)p.dg, p.m, p.n);
+  } else {
+    const int sb = block_rows > 0 ? block_rows : 1024;
+    const long long tiles = (p.rows + sb - 1) / sb;
+    const long long blocks = tiles * p.n_g;
+    if (blocks > 0x7fffffffLL) return GRKAN_ERR_SHAPE;
+    if (f32)
+      grk::bwd_atomic_block<grk::IoF32, GRKAN_MAX_M, GRKAN_MAX_N>
+          <<<(unsigned)blocks, grk::kAtomicThreads, 0, st>>>(
+              (const float*)x, (const float*)dy, (float*)dx, a, b, dA, dB, p.rows, p.d,
+              (int)p.dg, p.n_g, p.m, p.n, sb);
+    else
+      grk::bwd_atomic_block<grk::IoBF16, GRKAN_MAX_M, GRKAN_MAX_N>
+          <<<(unsigned)blocks, grk::kAtomicThreads, 0, st>>>(
+              (const grk::IoBF16::T*)x, (const grk::IoBF16::T*)dy, (grk::IoBF16::T*)dx, a, b,
+              dA, dB, p.rows, p.d, (int)p.dg, p.n_g, p.m, p.n, sb);
+  }
+  return cuda_status(cudaGetLastError(), "grkan_backward_atomic launch");
 }
 
 grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* dA, float* dB,

@@ -130,6 +130,30 @@ GRKAN_API grkan_status_t grkan_forward_backward(const void* x, const void* dy, c
                                                 size_t workspace_bytes, uint32_t flags,
                                                 void* stream);
 
+/* Coefficient gradients accumulated with float32 atomic adds, the two schemes
+ * that "FlashKAT: Understanding and Addressing Performance Bottlenecks in the
+ * Kolmogorov-Arnold Transformer" compares (paper notes, sections "2. The
+ * atomic-add problem of the original KAT" and "3. FlashKAT kernel restructuring
+ * (Algorithm 2)"), for error and speed studies against grkan_backward:
+ *   GRKAN_ATOMIC_PER_ELEMENT  every element adds its m+1+n terms to dA / dB in
+ *                             global memory (one thread per element);
+ *   GRKAN_ATOMIC_PER_BLOCK    a block sums block_rows rows of one group on chip,
+ *                             then adds each of its m+1+n sums once
+ *                             (block_rows = 0: 1024, the paper's typical S_block).
+ * dx is the same as grkan_backward's. dA and dB are zeroed on the stream first
+ * and then depend on the order in which the atomics land: they can differ from
+ * run to run. No workspace. Unknown mode: GRKAN_ERR_FLAGS. */
+typedef enum grkan_atomic_mode {
+  GRKAN_ATOMIC_PER_ELEMENT = 1,
+  GRKAN_ATOMIC_PER_BLOCK = 2
+} grkan_atomic_mode_t;
+
+GRKAN_API grkan_status_t grkan_backward_atomic(const void* x, const void* dy, const float* a,
+                                               const float* b, void* dx, float* dA, float* dB,
+                                               int64_t B, int64_t N, int64_t d, int32_t n_g,
+                                               int32_t m, int32_t n, grkan_dtype_t dtype,
+                                               int32_t mode, int32_t block_rows, void* stream);
+
 /* Stage 1 alone: dx, plus one float32 partial sum per (row tile, group,
  * coefficient) into the workspace. */
 GRKAN_API grkan_status_t grkan_backward_partials(const void* x, const void* dy, const float* a,
