@@ -52,8 +52,8 @@ struct TmaGeom {
 // One CTA of kWarps independent warps per SM. Every warp owns, per element
 // type, a ring of forward stages (one box of x each) and of backward stages
 // (one box of x and one of dy each). float32 rows are HBM-bound: smaller boxes,
-// deeper rings. The bf16 backward is bound by the FMA pipe: 3 KiB boxes read in
-// two passes of three 16-byte vectors per lane, two stages.
+// deeper rings. The bf16 backward is bound by arithmetic issue: 3 KiB boxes read
+// in three passes of two 16-byte vectors per lane, two stages.
 #ifndef GRK_WARPS
 #define GRK_WARPS 16
 #endif
@@ -62,6 +62,9 @@ struct TmaGeom {
 #endif
 #ifndef GRK_F32_FWD_STAGES
 #define GRK_F32_FWD_STAGES 4
+#endif
+#ifndef GRK_F32_BWD_VEC
+#define GRK_F32_BWD_VEC 3
 #endif
 #ifndef GRK_F32_BWD_HALVES
 #define GRK_F32_BWD_HALVES 1
@@ -75,8 +78,11 @@ struct TmaGeom {
 #ifndef GRK_BF16_FWD_STAGES
 #define GRK_BF16_FWD_STAGES 6
 #endif
+#ifndef GRK_BF16_BWD_VEC
+#define GRK_BF16_BWD_VEC 2
+#endif
 #ifndef GRK_BF16_BWD_HALVES
-#define GRK_BF16_BWD_HALVES 2
+#define GRK_BF16_BWD_HALVES 3
 #endif
 #ifndef GRK_BF16_BWD_STAGES
 #define GRK_BF16_BWD_STAGES 2
@@ -84,10 +90,6 @@ struct TmaGeom {
 
 constexpr int kWarps = GRK_WARPS;
 constexpr int kThreads = kWarps * 32;
-#ifndef GRK_BWD_VEC
-#define GRK_BWD_VEC 3
-#endif
-constexpr int kBwdVec = GRK_BWD_VEC;  // 16-byte vectors per lane and tensor in one backward pass
 
 template <class IO>
 struct Shape;
@@ -95,6 +97,7 @@ template <>
 struct Shape<IoF32> {
   static constexpr int kFwdVec = GRK_F32_FWD_VEC;        // vectors per lane in a forward box
   static constexpr int kFwdStages = GRK_F32_FWD_STAGES;  // forward ring depth
+  static constexpr int kBwdVec = GRK_F32_BWD_VEC;        // vectors per lane and tensor in one pass
   static constexpr int kBwdHalves = GRK_F32_BWD_HALVES;  // passes over a backward box
   static constexpr int kBwdStages = GRK_F32_BWD_STAGES;  // backward ring depth
 };
@@ -102,6 +105,7 @@ template <>
 struct Shape<IoBF16> {
   static constexpr int kFwdVec = GRK_BF16_FWD_VEC;
   static constexpr int kFwdStages = GRK_BF16_FWD_STAGES;
+  static constexpr int kBwdVec = GRK_BF16_BWD_VEC;
   static constexpr int kBwdHalves = GRK_BF16_BWD_HALVES;
   static constexpr int kBwdStages = GRK_BF16_BWD_STAGES;
 };
@@ -111,7 +115,7 @@ constexpr unsigned fwd_box_bytes() {
 }
 template <class IO>
 constexpr unsigned bwd_box_bytes() {
-  return 32u * kBwdVec * Shape<IO>::kBwdHalves * 16u;
+  return 32u * Shape<IO>::kBwdVec * Shape<IO>::kBwdHalves * 16u;
 }
 inline unsigned fwd_box_target(bool bf16) {
   return bf16 ? fwd_box_bytes<IoBF16>() : fwd_box_bytes<IoF32>();
@@ -592,6 +596,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
   using S_ = Shape<IO>;
   using T = typename IO::T;
+  constexpr int kBwdVec = S_::kBwdVec;
   constexpr int NV = kBwdVec * S_::kBwdHalves;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
@@ -621,26 +626,41 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   if (use_tab) build_coef_table(ctab, a, b, geom.n_g);
   __syncthreads();
 
-  // issue cursor (lane 0): unit (tile, g) = iu.hi, iu.lo; box (irb, ibx) of inrb row blocks
+  // issue cursor (lane 0): unit (tile, g) = iu.hi, iu.lo; box (irb, ibx) of inrb
+  // row blocks; the box origin (icol, irow) and the ring slot advance by addition
   Cursor3 iu;
   iu.init(gw, GW, 1, geom.n_g);
-  int irb = 0, ibx = 0, inrb = (iu.hi < geom.T) ? tile_row_blocks(geom, iu.hi) : 0;
+  int irb = 0, ibx = 0, inrb = 0, icol = 0, irow = 0, islot = 0;
   int iq = 0;
+  auto unit_start = [&]() {
+    if (iu.hi < geom.T) {
+      inrb = tile_row_blocks(geom, iu.hi);
+      icol = iu.lo * geom.dg;
+      irow = (int)(iu.hi * geom.S);
+    } else {
+      inrb = 0;
+    }
+  };
+  unit_start();
+  const uint32_t stage0 = smem_addr(base);
+  const uint32_t tx_bytes = 2u * geom.box_bytes;
   auto issue = [&]() {
-    const int s = iq % S_::kBwdStages;
-    const int col = iu.lo * geom.dg + ibx * geom.bw;
-    const int row = (int)(iu.hi * geom.S) + irb * geom.SCw;
-    unsigned char* st = base + s * L.stage;
-    mbar_arrive_expect_tx(full0 + 8 * s, 2u * geom.box_bytes);
-    tma_load_2d(smem_addr(st), &mx, col, row, full0 + 8 * s);
-    tma_load_2d(smem_addr(st + L.box_slot), &mdy, col, row, full0 + 8 * s);
+    const uint32_t bar = full0 + 8u * (uint32_t)islot;
+    const uint32_t dst = stage0 + (uint32_t)islot * L.stage;
+    mbar_arrive_expect_tx(bar, tx_bytes);
+    tma_load_2d(dst, &mx, icol, irow, bar);
+    tma_load_2d(dst + L.box_slot, &mdy, icol, irow, bar);
     ++iq;
+    islot = (islot + 1 == S_::kBwdStages) ? 0 : islot + 1;
+    icol += geom.bw;
     if (++ibx == geom.nbox) {
       ibx = 0;
+      icol -= geom.dg;  // nbox * bw == dg: back to the group's first column
+      irow += geom.SCw;
       if (++irb == inrb) {
         irb = 0;
         iu.next();
-        inrb = (iu.hi < geom.T) ? tile_row_blocks(geom, iu.hi) : 0;
+        unit_start();
       }
     }
   };
@@ -659,7 +679,8 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   int cur_g = -1;
   Acc54 acc;
   bool ok = true;
-  int q = 0;
+  int q = 0, rslot = 0;  // boxes consumed; ring slot and phase of the next one
+  uint32_t rphase = 0;
   Cursor3 cu;
   cu.init(gw, GW, 1, geom.n_g);
   for (; cu.hi < geom.T && ok; cu.next()) {
@@ -681,8 +702,12 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
       const int r0 = rb * geom.SCw;     // row of the box within the tile
       const int lim = rows_left - r0;   // lane vectors in rows >= lim are past the end
       for (int bx = 0; bx < geom.nbox; ++bx, ++q) {
-        const int s = q % S_::kBwdStages;
-        const uint32_t ph = (uint32_t)(q / S_::kBwdStages) & 1;
+        const int s = rslot;
+        const uint32_t ph = rphase;
+        if (++rslot == S_::kBwdStages) {
+          rslot = 0;
+          rphase ^= 1u;
+        }
         if (!mbar_wait(full0 + 8 * s, ph)) {
           report(kErrFullWait);
           ok = false;
@@ -863,7 +888,7 @@ inline cudaError_t launch_bwd_tma_io(const TmaGeom& g, const CUtensorMap& mx,
                                      const CUtensorMap& mdy, void* dx, void* y, const float* a,
                                      const float* b, float* ws, long long grid, cudaStream_t st) {
   // every lane vector slot used: the box is exactly 32 lanes x NV vectors
-  const bool full = g.box_bytes == 16u * 32u * (unsigned)(kBwdVec * Shape<IO>::kBwdHalves);
+  const bool full = g.box_bytes == bwd_box_bytes<IO>();
   if (full)
     return y ? launch_bwd_tma_t<IO, true, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
              : launch_bwd_tma_t<IO, false, true>(g, mx, mdy, dx, y, a, b, ws, grid, st);
