@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--ng", type=int, default=None, help="groups for the stress workload")
     ap.add_argument("--rows", type=int, default=None,
                     help="use only the first ROWS rows of the workload (profiling captures)")
+    ap.add_argument("--m", type=int, default=None, help="numerator degree (degree sweeps)")
+    ap.add_argument("--n", type=int, default=None, help="denominator degree (degree sweeps)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
@@ -206,6 +208,10 @@ def main():
         w = w.with_rows(args.rows)
         w.B, w.N = args.rows, 1
         w.rows_override = None
+    if args.m is not None:
+        w.m = args.m
+    if args.n is not None:
+        w.n = args.n
     if args.impl == "reference":
         return run_reference(args, w)
 

@@ -334,7 +334,8 @@ grkan_status_t do_partials_at(const Plan& p, const void* x, const void* dy, cons
                               const float* b, void* dx, void* y, void* ws, long long ws_T,
                               long long tile0, uint32_t flags, cudaStream_t st) {
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
-  if (choose_bwd_path(p, x, dy, dx, flags) == 1 && (!y || aligned16(y)))
+  if (choose_bwd_path(p, x, dy, dx, flags) == 1 &&
+      (!y || (aligned16(y) && grk::tma_has_fused_degree(p.m, p.n))))
     return launch_tma_bwd(p, x, dy, dx, y, a, b, (float*)ws, ws_T, tile0, st);
   if (y) {
     cudaError_t e = (p.dtype == GRKAN_F32) ? launch_generic_fwd<grk::IoF32>(p, x, y, a, b, st)

@@ -137,7 +137,20 @@ constexpr unsigned kErrDrainWait = 8u;
 
 __device__ unsigned int g_grkan_device_error = 0;
 
-inline bool tma_has_degree(int m, int n) { return m == 5 && n == 4; }
+// Degrees (m, n) with TMA-pipelined kernels: the KAT degree (5, 4) and m = n
+// from 3 to 8 (for degree sweeps); every other degree takes the generic kernels.
+#define GRK_TMA_DEGREES(X) X(3, 3) X(4, 4) X(5, 4) X(5, 5) X(6, 6) X(7, 7) X(8, 8)
+
+inline bool tma_has_degree(int m, int n) {
+#define GRK_DEG_CASE(M, N) \
+  if (m == M && n == N) return true;
+  GRK_TMA_DEGREES(GRK_DEG_CASE)
+#undef GRK_DEG_CASE
+  return false;
+}
+// The forward-and-backward (recompute) variant of the backward kernel exists for
+// the KAT degree only.
+inline bool tma_has_fused_degree(int m, int n) { return m == 5 && n == 4; }
 
 // --- PTX wrappers --------------------------------------------------------------
 
@@ -229,12 +242,6 @@ struct Coef54 {
   float2 b1, b2, b3, b4;              // b_j
   float2 jb2, jb3, jb4;               // j * b_j  (Q')
 
-  __device__ __forceinline__ void set(const float* c) {  // c = a_0..a_5, b_1..b_4
-    a0 = f2(c[0]); a1 = f2(c[1]); a2 = f2(c[2]); a3 = f2(c[3]); a4 = f2(c[4]); a5 = f2(c[5]);
-    ia2 = f2(2.f * c[2]); ia3 = f2(3.f * c[3]); ia4 = f2(4.f * c[4]); ia5 = f2(5.f * c[5]);
-    b1 = f2(c[6]); b2 = f2(c[7]); b3 = f2(c[8]); b4 = f2(c[9]);
-    jb2 = f2(2.f * c[7]); jb3 = f2(3.f * c[8]); jb4 = f2(4.f * c[9]);
-  }
 };
 
 // y for a pair of elements: Horner for P and for Q / x.
@@ -295,6 +302,197 @@ __host__ __device__ constexpr unsigned round_up(unsigned v, unsigned a) {
   return (v + a - 1) / a * a;
 }
 
+// --- degree traits ------------------------------------------------------------------
+//
+// Deg<M, N> gives the packed kernels their coefficient registers, sums and
+// per-pair arithmetic. The generic form evaluates in the power basis (x^k by
+// balanced products, then one FMA per term); Deg<5, 4> is the hand-scheduled
+// Estrin form above.
+
+// Floats per group in the coefficient table: a_0..a_M, i a_i (i = 2..M),
+// b_1..b_N, j b_j (j = 2..N), padded to a multiple of four.
+template <int M, int N>
+__host__ __device__ constexpr int tab_floats() {
+  return ((M + 1) + (M - 1) + N + (N - 1) + 3) / 4 * 4;
+}
+
+// Table entry k of group g (the layout above), from the coefficient arrays.
+template <int M, int N>
+__device__ __forceinline__ float coef_value(const float* a, const float* b, int g, int k) {
+  if (k <= M) return __ldg(a + g * (M + 1) + k);
+  if (k < 2 * M) {
+    const int i = k - (M + 1) + 2;
+    return (float)i * __ldg(a + g * (M + 1) + i);
+  }
+  if (k < 2 * M + N) return __ldg(b + g * N + (k - 2 * M));
+  if (k < 2 * M + 2 * N - 1) {
+    const int j = k - (2 * M + N) + 2;
+    return (float)j * __ldg(b + g * N + (j - 1));
+  }
+  return 0.f;
+}
+
+template <int M, int N>
+struct Deg {
+  static constexpr int K = M + 1 + N;
+  static constexpr int TF = tab_floats<M, N>();
+  struct Coef {
+    float2 a[M + 1];   // a_i
+    float2 ia[M + 1];  // i a_i, i >= 2
+    float2 b[N + 1];   // b_j, j >= 1
+    float2 jb[N + 1];  // j b_j, j >= 2
+  };
+  struct Acc {
+    float2 a[M + 1], b[N];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+      for (int i = 0; i <= M; ++i) a[i] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < N; ++j) b[j] = make_float2(0.f, 0.f);
+    }
+  };
+  __device__ static __forceinline__ void assign(const float (&v)[TF], Coef& c) {
+    int o = 0;
+#pragma unroll
+    for (int i = 0; i <= M; ++i) c.a[i] = f2(v[o++]);
+#pragma unroll
+    for (int i = 2; i <= M; ++i) c.ia[i] = f2(v[o++]);
+#pragma unroll
+    for (int j = 1; j <= N; ++j) c.b[j] = f2(v[o++]);
+#pragma unroll
+    for (int j = 2; j <= N; ++j) c.jb[j] = f2(v[o++]);
+  }
+  __device__ static __forceinline__ float2 fwd(const Coef& c, float2 x) {
+    float2 P = c.a[M];
+#pragma unroll
+    for (int i = M - 1; i >= 0; --i) P = fma2(P, x, c.a[i]);
+    float2 q = c.b[N];
+#pragma unroll
+    for (int j = N - 1; j >= 1; --j) q = fma2(q, x, c.b[j]);
+    const float2 Q = mul2(q, x);
+    const float2 r = make_float2(rcp_approx(1.f + fabsf(Q.x)), rcp_approx(1.f + fabsf(Q.y)));
+    return mul2(P, r);
+  }
+  __device__ static __forceinline__ float2 bwd(const Coef& c, float2 x, float2 dy, Acc& acc,
+                                               float2* y_out) {
+    constexpr int KP = M > N ? M : N;
+    float2 p[KP + 1];  // p[k] = x^k
+    p[1] = x;
+#pragma unroll
+    for (int k = 2; k <= KP; ++k) p[k] = mul2(p[k / 2], p[k - k / 2]);
+    float2 P = fma2(c.a[1], x, c.a[0]);
+#pragma unroll
+    for (int i = 2; i <= M; ++i) P = fma2(c.a[i], p[i], P);
+    float2 dP = c.a[1];
+#pragma unroll
+    for (int i = 2; i <= M; ++i) dP = fma2(c.ia[i], p[i - 1], dP);
+    float2 Q = mul2(c.b[1], x);
+#pragma unroll
+    for (int j = 2; j <= N; ++j) Q = fma2(c.b[j], p[j], Q);
+    float2 dQ = c.b[1];
+#pragma unroll
+    for (int j = 2; j <= N; ++j) dQ = fma2(c.jb[j], p[j - 1], dQ);
+    const float2 r = make_float2(rcp_approx(1.f + fabsf(Q.x)), rcp_approx(1.f + fabsf(Q.y)));
+    const float2 y = mul2(P, r);
+    if (y_out) *y_out = y;
+    const float2 t = mul2(dy, r);
+    const float2 nu = mul2(t, make_float2(neg_y_sign(y.x, Q.x), neg_y_sign(y.y, Q.y)));
+    acc.a[0] = add2(acc.a[0], t);
+#pragma unroll
+    for (int i = 1; i <= M; ++i) acc.a[i] = fma2(t, p[i], acc.a[i]);
+#pragma unroll
+    for (int j = 1; j <= N; ++j) acc.b[j - 1] = fma2(nu, p[j], acc.b[j - 1]);
+    return fma2(nu, dQ, mul2(t, dP));
+  }
+  template <int NS>
+  __device__ static __forceinline__ void sums(const Acc& acc, float (&v)[NS]) {
+#pragma unroll
+    for (int i = 0; i <= M; ++i) v[i] = acc.a[i].x + acc.a[i].y;
+#pragma unroll
+    for (int j = 0; j < N; ++j) v[M + 1 + j] = acc.b[j].x + acc.b[j].y;
+#pragma unroll
+    for (int k = K; k < NS; ++k) v[k] = 0.f;
+  }
+};
+
+template <>
+struct Deg<5, 4> {
+  static constexpr int K = 10;
+  static constexpr int TF = tab_floats<5, 4>();
+  using Coef = Coef54;
+  using Acc = Acc54;
+  __device__ static __forceinline__ void assign(const float (&v)[TF], Coef54& c) {
+    c.a0 = f2(v[0]); c.a1 = f2(v[1]); c.a2 = f2(v[2]); c.a3 = f2(v[3]);
+    c.a4 = f2(v[4]); c.a5 = f2(v[5]); c.ia2 = f2(v[6]); c.ia3 = f2(v[7]);
+    c.ia4 = f2(v[8]); c.ia5 = f2(v[9]); c.b1 = f2(v[10]); c.b2 = f2(v[11]);
+    c.b3 = f2(v[12]); c.b4 = f2(v[13]); c.jb2 = f2(v[14]); c.jb3 = f2(v[15]);
+    c.jb4 = f2(v[16]);
+  }
+  __device__ static __forceinline__ float2 fwd(const Coef54& c, float2 x) { return fwd_pair(c, x); }
+  __device__ static __forceinline__ float2 bwd(const Coef54& c, float2 x, float2 dy, Acc54& acc,
+                                               float2* y_out) {
+    return bwd_pair(c, x, dy, acc, y_out);
+  }
+  template <int NS>
+  __device__ static __forceinline__ void sums(const Acc54& acc, float (&v)[NS]) {
+    v[0] = acc.a0.x + acc.a0.y;
+    v[1] = acc.a1.x + acc.a1.y;
+    v[2] = acc.a2.x + acc.a2.y;
+    v[3] = acc.a3.x + acc.a3.y;
+    v[4] = acc.a4.x + acc.a4.y;
+    v[5] = acc.a5.x + acc.a5.y;
+    v[6] = acc.b1.x + acc.b1.y;
+    v[7] = acc.b2.x + acc.b2.y;
+    v[8] = acc.b3.x + acc.b3.y;
+    v[9] = acc.b4.x + acc.b4.y;
+#pragma unroll
+    for (int k = 10; k < NS; ++k) v[k] = 0.f;
+  }
+};
+
+// Coefficients of every group in the CTA's shared memory after the warps'
+// regions (tab_floats per group), used when n_g <= kTableGroups; with more
+// groups every lane reads its group's entries from global memory (broadcast
+// loads). Scalars, not pairs: a pair built in registers from one scalar lets the
+// compiler keep one register per coefficient.
+constexpr int kTableGroups = 64;
+template <int M, int N>
+__host__ __device__ constexpr unsigned coef_table_bytes() {
+  return (unsigned)(kTableGroups * tab_floats<M, N>() * 4);
+}
+
+template <int M, int N>
+__device__ __forceinline__ void build_coef_table(float* tab, const float* a, const float* b,
+                                                 int n_g) {
+  constexpr int TF = tab_floats<M, N>();
+  for (int e = threadIdx.x; e < n_g * TF; e += blockDim.x) {
+    const int g = e / TF;
+    tab[e] = coef_value<M, N>(a, b, g, e - g * TF);
+  }
+}
+
+template <int M, int N>
+__device__ __forceinline__ void load_coef(bool use_tab, const float* tab, const float* a,
+                                          const float* b, int g, typename Deg<M, N>::Coef& c) {
+  using D = Deg<M, N>;
+  float v[D::TF];
+  if (use_tab) {
+    const float4* q = reinterpret_cast<const float4*>(tab + g * D::TF);
+#pragma unroll
+    for (int k = 0; k < D::TF / 4; ++k) {
+      const float4 w = q[k];
+      v[4 * k] = w.x;
+      v[4 * k + 1] = w.y;
+      v[4 * k + 2] = w.z;
+      v[4 * k + 3] = w.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < D::TF; ++k) v[k] = coef_value<M, N>(a, b, g, k);
+  }
+  D::assign(v, c);
+}
+
 // --- per-warp pipeline geometry ----------------------------------------------------
 //
 // Every warp runs its own pipeline: it owns kStages stage slots in shared
@@ -303,21 +501,17 @@ __host__ __device__ constexpr unsigned round_up(unsigned v, unsigned a) {
 // CTA after initialisation, so they drift out of phase and one warp's loads
 // and reductions overlap another's arithmetic.
 
-constexpr int kCoefFloats = 16;  // per-warp coefficient slot (10 used)
-
-// Per-warp shared memory: [stages][tensors][box, 128-byte rounded],
-// coefficient slot, then the 8-byte barriers.
+// Per-warp shared memory: [stages][tensors][box, 128-byte rounded], then the
+// 8-byte barriers.
 struct WarpLayout {
   unsigned box_slot;   // bytes of one box slot
   unsigned stage;      // bytes of one stage (all tensors)
-  unsigned coef_off;   // coefficient slot
   unsigned bar_off;    // full[stages] then empty[stages]
   unsigned per_warp;   // bytes per warp (multiple of 128)
   __host__ __device__ WarpLayout(unsigned box_bytes, int tensors, int stages) {
     box_slot = round_up(box_bytes, 128);
     stage = box_slot * (unsigned)tensors;
-    coef_off = stage * (unsigned)stages;
-    bar_off = coef_off + kCoefFloats * 4;
+    bar_off = stage * (unsigned)stages;
     per_warp = round_up(bar_off + (unsigned)(2 * stages) * 8, 128);
   }
 };
@@ -352,26 +546,19 @@ __device__ __forceinline__ void store16(void* p, uint4 v) {
   __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
-// Stage a group's coefficients a_0..a_5, b_1..b_4 in the warp's shared slot
-// and read them back on every lane.
-__device__ __forceinline__ void stage_coefficients(float* slot, const float* a, const float* b,
-                                                   int g, int lane, Coef54& c) {
-  if (lane < 6) slot[lane] = __ldg(a + g * 6 + lane);
-  else if (lane < 10) slot[lane] = __ldg(b + g * 4 + (lane - 6));
-  __syncwarp();
-  c.set(slot);
-  __syncwarp();
-}
-
-// Sum ten per-lane values over the warp in a fixed order; every lane ends with
-// all ten sums. Recursive halving: at each step a lane keeps half of its
-// values (those of its own half of the index range) and adds the partner's.
-__device__ __forceinline__ void warp_sum10(float (&v)[16], int lane) {
-  // 16 slots, 10 used (the rest are zero)
+// Sum NS (16 or 32) per-lane values over the warp in a fixed order.
+// Recursive halving: at each step a lane keeps half of its values (those of its
+// own half of the index range) and adds the partner's. Afterwards lane l holds
+// in v[0] the sum of value (l >> 1) & 15 (NS = 16: the last step adds the two
+// lanes of a pair) or of value l (NS = 32).
+template <int NS>
+__device__ __forceinline__ void warp_sum(float (&v)[NS], int lane) {
+  static_assert(NS == 16 || NS == 32, "16 or 32 slots");
+  constexpr int kSteps = NS == 16 ? 4 : 5;
 #pragma unroll
-  for (int step = 0; step < 4; ++step) {
-    const int half = 8 >> step;       // values kept after this step
-    const int mask = 16 >> step;      // partner distance
+  for (int step = 0; step < kSteps; ++step) {
+    const int half = (NS / 2) >> step;  // values kept after this step
+    const int mask = 16 >> step;        // partner distance
     const bool upper = (lane & mask) != 0;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
@@ -380,8 +567,7 @@ __device__ __forceinline__ void warp_sum10(float (&v)[16], int lane) {
       v[i] = (upper ? v[i + half] : v[i]) + recv;
     }
   }
-  // now lane holds, in v[0], the sum over lanes l with l & 1 == lane & 1 ...
-  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+  if constexpr (NS == 16) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 // Mixed-radix counter (hi, mid, lo) with radices (unbounded, nmid, nlo), stepped
@@ -420,17 +606,19 @@ struct Cursor3 {
 // grid as item gw, gw + total warps, ... in row-block-major order.
 
 
-template <class IO>
+template <class IO, int M, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
   using S_ = Shape<IO>;
+  using D = Deg<M, N>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const WarpLayout L(geom.box_bytes, 1, S_::kFwdStages);
   unsigned char* base = smem + warp * L.per_warp;
-  float* cslot = reinterpret_cast<float*>(base + L.coef_off);
+  float* ctab = reinterpret_cast<float*>(smem + kWarps * L.per_warp);
+  const bool use_tab = geom.n_g <= kTableGroups;
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * S_::kFwdStages;
   const long long row_blocks = (geom.rows + geom.SCw - 1) / geom.SCw;
@@ -446,7 +634,8 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     fence_proxy_async_smem();
     if (warp == 0) prefetch_map(&mx);
   }
-  __syncwarp();
+  if (use_tab) build_coef_table<M, N>(ctab, a, b, geom.n_g);
+  __syncthreads();
 
   Cursor3 ic;  // issue cursor (lane 0): (row block, group, box)
   ic.init(gw, GW, geom.n_g, geom.nbox);
@@ -465,7 +654,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
 
   LaneMap<IO, S_::kFwdVec> lm;
   lm.init(geom, lane, geom.d);
-  Coef54 c;
+  typename D::Coef c;
   int cur_g = -1;
   bool ok = true;
   int q = 0;
@@ -481,7 +670,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     }
     const int g = cc.mid;
     if (g != cur_g) {
-      stage_coefficients(cslot, a, b, g, lane, c);
+      load_coef<M, N>(use_tab, ctab, a, b, g, c);
       cur_g = g;
     }
     const uint4* buf = reinterpret_cast<const uint4*>(base + s * L.stage);
@@ -509,15 +698,15 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
       if (row0 + lm.row[it] < geom.rows) {
         uint4 o;
         if constexpr (IO::kBytes == 2) {
-          o.x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].x)));
-          o.y = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].y)));
-          o.z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].z)));
-          o.w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[it].w)));
+          o.x = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].x)));
+          o.y = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].y)));
+          o.z = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].z)));
+          o.w = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].w)));
         } else {
           const float2 p0 =
-              fwd_pair(c, make_float2(__uint_as_float(v[it].x), __uint_as_float(v[it].y)));
+              D::fwd(c, make_float2(__uint_as_float(v[it].x), __uint_as_float(v[it].y)));
           const float2 p1 =
-              fwd_pair(c, make_float2(__uint_as_float(v[it].z), __uint_as_float(v[it].w)));
+              D::fwd(c, make_float2(__uint_as_float(v[it].z), __uint_as_float(v[it].w)));
           o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
                          __float_as_uint(p1.y));
         }
@@ -548,47 +737,11 @@ __device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile)
   return tile == g.T - 1 ? g.nrb_last : g.nrb_full;
 }
 
-// Coefficients of every group in the CTA's shared memory after the warps'
-// regions, 20 floats per group (a_0..a_5, i a_i for i = 2..5, b_1..b_4, j b_j for
-// j = 2..4, padding), used when n_g <= kTableGroups; larger group counts stage
-// one group at a time in the warp's own slot. Scalars, not pairs: a pair built
-// in registers from one scalar lets the compiler keep one register per
-// coefficient.
-constexpr int kTableGroups = 64;
-constexpr int kTabFloats = 20;
-__host__ __device__ constexpr unsigned coef_table_bytes() {
-  return (unsigned)(kTableGroups * kTabFloats * 4);
-}
-
-__device__ __forceinline__ void build_coef_table(float* tab, const float* a, const float* b,
-                                                 int n_g) {
-  for (int e = threadIdx.x; e < n_g * kTabFloats; e += blockDim.x) {
-    const int g = e / kTabFloats;
-    const int k = e - g * kTabFloats;
-    float v = 0.f;
-    if (k < 6) v = __ldg(a + g * 6 + k);                                  // a_0..a_5
-    else if (k < 10) v = (float)(k - 4) * __ldg(a + g * 6 + (k - 4));    // i a_i, i = 2..5
-    else if (k < 14) v = __ldg(b + g * 4 + (k - 10));                    // b_1..b_4
-    else if (k < 17) v = (float)(k - 12) * __ldg(b + g * 4 + (k - 13));  // j b_j, j = 2..4
-    tab[e] = v;
-  }
-}
-
-__device__ __forceinline__ void load_coef(const float* t, Coef54& c) {
-  const float4* q = reinterpret_cast<const float4*>(t);
-  const float4 v0 = q[0], v1 = q[1], v2 = q[2], v3 = q[3], v4 = q[4];
-  c.a0 = f2(v0.x); c.a1 = f2(v0.y); c.a2 = f2(v0.z); c.a3 = f2(v0.w);
-  c.a4 = f2(v1.x); c.a5 = f2(v1.y); c.ia2 = f2(v1.z); c.ia3 = f2(v1.w);
-  c.ia4 = f2(v2.x); c.ia5 = f2(v2.y); c.b1 = f2(v2.z); c.b2 = f2(v2.w);
-  c.b3 = f2(v3.x); c.b4 = f2(v3.y); c.jb2 = f2(v3.z); c.jb3 = f2(v3.w);
-  c.jb4 = f2(v4.x);
-}
-
 // kWithY: also write y (the forward output recomputed on the way), for
 // training that recomputes the activation during the backward pass.
 // kFull: every 16-byte vector slot of a lane holds box data (the box is exactly
 // 32 * NV vectors), so the loads need no guard.
-template <class IO, bool kWithY, bool kFull>
+template <class IO, int M, int N, bool kWithY, bool kFull>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
         typename IO::T* __restrict__ dx, typename IO::T* __restrict__ yout,
@@ -596,14 +749,16 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
   using S_ = Shape<IO>;
   using T = typename IO::T;
-  constexpr int kBwdVec = S_::kBwdVec;
-  constexpr int NV = kBwdVec * S_::kBwdHalves;
+  using D = Deg<M, N>;
+  constexpr int NV = S_::kBwdVec * S_::kBwdHalves;  // 16-byte vectors per lane in a box
+  // vectors per pass: fewer for high degrees, whose per-pair state is larger
+  constexpr int kBwdVec = (M + N > 9) ? 1 : S_::kBwdVec;
+  constexpr int kPasses = NV / kBwdVec;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const WarpLayout L(geom.box_bytes, 2, S_::kBwdStages);
   unsigned char* base = smem + warp * L.per_warp;
-  float* cslot = reinterpret_cast<float*>(base + L.coef_off);
   float* ctab = reinterpret_cast<float*>(smem + kWarps * L.per_warp);
   const bool use_tab = geom.n_g <= kTableGroups;
   const uint32_t full0 = smem_addr(base + L.bar_off);
@@ -623,7 +778,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
       prefetch_map(&mdy);
     }
   }
-  if (use_tab) build_coef_table(ctab, a, b, geom.n_g);
+  if (use_tab) build_coef_table<M, N>(ctab, a, b, geom.n_g);
   __syncthreads();
 
   // issue cursor (lane 0): unit (tile, g) = iu.hi, iu.lo; box (irb, ibx) of inrb
@@ -675,9 +830,9 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 #pragma unroll
   for (int sl = 0; sl < NV; ++sl) boff[sl] = lm.off[sl] * (int)sizeof(T);
   const long long row_bytes = geom.d * (long long)sizeof(T);
-  Coef54 c;
+  typename D::Coef c;
   int cur_g = -1;
-  Acc54 acc;
+  typename D::Acc acc;
   bool ok = true;
   int q = 0, rslot = 0;  // boxes consumed; ring slot and phase of the next one
   uint32_t rphase = 0;
@@ -688,8 +843,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     const int g = cu.lo;
     const int nrb = tile_row_blocks(geom, tile);
     if (g != cur_g) {
-      if (use_tab) load_coef(ctab + g * kTabFloats, c);
-      else stage_coefficients(cslot, a, b, g, lane, c);
+      load_coef<M, N>(use_tab, ctab, a, b, g, c);
       cur_g = g;
     }
     acc.zero();
@@ -719,7 +873,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         char* dxo = dxt + box_off;
         char* yo = kWithY ? yt + box_off : nullptr;
 #pragma unroll
-        for (int h = 0; h < S_::kBwdHalves; ++h) {
+        for (int h = 0; h < kPasses; ++h) {
           uint4 xv[kBwdVec], gv[kBwdVec];
 #pragma unroll
           for (int it = 0; it < kBwdVec; ++it) {
@@ -732,7 +886,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
               gv[it] = make_uint4(0, 0, 0, 0);
             }
           }
-          if (h == S_::kBwdHalves - 1) {
+          if (h == kPasses - 1) {
             // release the slot (every lane has read it) and refill it
             __syncwarp();
             if (lane == 0) {
@@ -756,22 +910,22 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
             float2 y0, y1, y2, y3;
             if constexpr (IO::kBytes == 2) {
               o.x = f2_to_bf16x2(
-                  bwd_pair(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc, kWithY ? &y0 : nullptr));
+                  D::bwd(c, bf16x2_to_f2(xv[it].x), bf16x2_to_f2(gv[it].x), acc, kWithY ? &y0 : nullptr));
               o.y = f2_to_bf16x2(
-                  bwd_pair(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc, kWithY ? &y1 : nullptr));
+                  D::bwd(c, bf16x2_to_f2(xv[it].y), bf16x2_to_f2(gv[it].y), acc, kWithY ? &y1 : nullptr));
               o.z = f2_to_bf16x2(
-                  bwd_pair(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc, kWithY ? &y2 : nullptr));
+                  D::bwd(c, bf16x2_to_f2(xv[it].z), bf16x2_to_f2(gv[it].z), acc, kWithY ? &y2 : nullptr));
               o.w = f2_to_bf16x2(
-                  bwd_pair(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc, kWithY ? &y3 : nullptr));
+                  D::bwd(c, bf16x2_to_f2(xv[it].w), bf16x2_to_f2(gv[it].w), acc, kWithY ? &y3 : nullptr));
               if constexpr (kWithY)
                 oy = make_uint4(f2_to_bf16x2(y0), f2_to_bf16x2(y1), f2_to_bf16x2(y2),
                                 f2_to_bf16x2(y3));
             } else {
-              const float2 p0 = bwd_pair(
+              const float2 p0 = D::bwd(
                   c, make_float2(__uint_as_float(xv[it].x), __uint_as_float(xv[it].y)),
                   make_float2(__uint_as_float(gv[it].x), __uint_as_float(gv[it].y)), acc,
                   kWithY ? &y0 : nullptr);
-              const float2 p1 = bwd_pair(
+              const float2 p1 = D::bwd(
                   c, make_float2(__uint_as_float(xv[it].z), __uint_as_float(xv[it].w)),
                   make_float2(__uint_as_float(gv[it].z), __uint_as_float(gv[it].w)), acc,
                   kWithY ? &y1 : nullptr);
@@ -794,24 +948,13 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     if (!ok) break;
     // Unit reduction, fixed order: the two lanes of each pair, then a
     // recursive-halving exchange over the warp.
-    float v[16];
-    v[0] = acc.a0.x + acc.a0.y;
-    v[1] = acc.a1.x + acc.a1.y;
-    v[2] = acc.a2.x + acc.a2.y;
-    v[3] = acc.a3.x + acc.a3.y;
-    v[4] = acc.a4.x + acc.a4.y;
-    v[5] = acc.a5.x + acc.a5.y;
-    v[6] = acc.b1.x + acc.b1.y;
-    v[7] = acc.b2.x + acc.b2.y;
-    v[8] = acc.b3.x + acc.b3.y;
-    v[9] = acc.b4.x + acc.b4.y;
-#pragma unroll
-    for (int k = 10; k < 16; ++k) v[k] = 0.f;
-    warp_sum10(v, lane);
-    // after the exchange lane l holds the sum of coefficient (l >> 1) & 15
-    const int k = (lane >> 1) & 15;
-    if ((lane & 1) == 0 && k < 10)
-      ws[((long long)g * 10 + k) * geom.ws_T + geom.ws_tile0 + tile] = v[0];
+    constexpr int NS = D::K <= 16 ? 16 : 32;
+    float v[NS];
+    D::template sums<NS>(acc, v);
+    warp_sum<NS>(v, lane);
+    const int k = NS == 16 ? ((lane >> 1) & 15) : lane;
+    if ((NS == 32 || (lane & 1) == 0) && k < D::K)
+      ws[((long long)g * D::K + k) * geom.ws_T + geom.ws_tile0 + tile] = v[0];
   }
   if (!ok && lane == 0) {
     for (int j = q; j < iq; ++j)
@@ -841,15 +984,28 @@ inline cudaError_t ensure_smem(unsigned bytes) {
   return e;
 }
 
-// Shared memory of a launch: kWarps per-warp regions of the largest box.
-template <class IO>
+// Shared memory of a launch: kWarps per-warp regions of the largest box, then
+// the coefficient table.
+template <class IO, int M, int N>
 inline unsigned fwd_smem_bytes() {
-  return kWarps * WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages).per_warp;
+  return kWarps * WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages).per_warp +
+         coef_table_bytes<M, N>();
 }
-template <class IO>
+template <class IO, int M, int N>
 inline unsigned bwd_smem_bytes() {
   return kWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp +
-         coef_table_bytes();
+         coef_table_bytes<M, N>();
+}
+
+template <class IO, int M, int N>
+inline cudaError_t launch_fwd_tma_t(const TmaGeom& g, const CUtensorMap& mx, void* y,
+                                    const float* a, const float* b, long long grid,
+                                    cudaStream_t st) {
+  const unsigned smem = fwd_smem_bytes<IO, M, N>();
+  cudaError_t e = ensure_smem<fwd_tma<IO, M, N>>(smem);
+  if (e != cudaSuccess) return e;
+  fwd_tma<IO, M, N><<<(unsigned)grid, kThreads, smem, st>>>(mx, (typename IO::T*)y, a, b, g);
+  return cudaGetLastError();
 }
 
 inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx, void* y,
@@ -858,45 +1014,47 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   const long long items = ((g.rows + g.SCw - 1) / g.SCw) * g.n_g * g.nbox;
   long long grid = sms;
   if (grid * kWarps > items) grid = (items + kWarps - 1) / kWarps;
-  cudaError_t e;
-  if (bf16) {
-    const unsigned smem = fwd_smem_bytes<IoBF16>();
-    if ((e = ensure_smem<fwd_tma<IoBF16>>(smem)) != cudaSuccess) return e;
-    fwd_tma<IoBF16><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoBF16::T*)y, a, b, g);
-  } else {
-    const unsigned smem = fwd_smem_bytes<IoF32>();
-    if ((e = ensure_smem<fwd_tma<IoF32>>(smem)) != cudaSuccess) return e;
-    fwd_tma<IoF32><<<(unsigned)grid, kThreads, smem, st>>>(mx, (IoF32::T*)y, a, b, g);
-  }
-  return cudaGetLastError();
+#define GRK_FWD_CASE(M, N)                                                          \
+  if (g.m == M && g.n == N)                                                         \
+    return bf16 ? launch_fwd_tma_t<IoBF16, M, N>(g, mx, y, a, b, grid, st)          \
+                : launch_fwd_tma_t<IoF32, M, N>(g, mx, y, a, b, grid, st);
+  GRK_TMA_DEGREES(GRK_FWD_CASE)
+#undef GRK_FWD_CASE
+  return cudaErrorNotSupported;
 }
 
-template <class IO, bool kWithY, bool kFull>
+template <class IO, int M, int N, bool kWithY, bool kFull>
 inline cudaError_t launch_bwd_tma_t(const TmaGeom& g, const CUtensorMap& mx,
                                     const CUtensorMap& mdy, void* dx, void* y, const float* a,
                                     const float* b, float* ws, long long grid, cudaStream_t st) {
-  const unsigned smem = bwd_smem_bytes<IO>();
-  cudaError_t e = ensure_smem<bwd_tma<IO, kWithY, kFull>>(smem);
+  const unsigned smem = bwd_smem_bytes<IO, M, N>();
+  cudaError_t e = ensure_smem<bwd_tma<IO, M, N, kWithY, kFull>>(smem);
   if (e != cudaSuccess) return e;
-  bwd_tma<IO, kWithY, kFull><<<(unsigned)grid, kThreads, smem, st>>>(
+  bwd_tma<IO, M, N, kWithY, kFull><<<(unsigned)grid, kThreads, smem, st>>>(
       mx, mdy, (typename IO::T*)dx, (typename IO::T*)y, a, b, ws, g);
   return cudaGetLastError();
 }
 
-template <class IO>
+template <class IO, int M, int N>
 inline cudaError_t launch_bwd_tma_io(const TmaGeom& g, const CUtensorMap& mx,
                                      const CUtensorMap& mdy, void* dx, void* y, const float* a,
                                      const float* b, float* ws, long long grid, cudaStream_t st) {
   // every lane vector slot used: the box is exactly 32 lanes x NV vectors
   const bool full = g.box_bytes == bwd_box_bytes<IO>();
-  if (full)
-    return y ? launch_bwd_tma_t<IO, true, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-             : launch_bwd_tma_t<IO, false, true>(g, mx, mdy, dx, y, a, b, ws, grid, st);
-  return y ? launch_bwd_tma_t<IO, true, false>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-           : launch_bwd_tma_t<IO, false, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+  if (y) {
+    if constexpr (M == 5 && N == 4) {
+      return full ? launch_bwd_tma_t<IO, M, N, true, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+                  : launch_bwd_tma_t<IO, M, N, true, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+    } else {
+      return cudaErrorNotSupported;
+    }
+  }
+  return full ? launch_bwd_tma_t<IO, M, N, false, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
+              : launch_bwd_tma_t<IO, M, N, false, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
 }
 
-// y == nullptr: backward only; otherwise also write the recomputed forward y.
+// y == nullptr: backward only; otherwise also write the recomputed forward y
+// (degree (5, 4) only).
 inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
                                   const CUtensorMap& mdy, void* dx, void* y, const float* a,
                                   const float* b, float* ws, int sms, cudaStream_t st) {
@@ -904,8 +1062,13 @@ inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   const long long units = g.T * g.n_g;
   long long grid = sms;
   if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
-  return bf16 ? launch_bwd_tma_io<IoBF16>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-              : launch_bwd_tma_io<IoF32>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+#define GRK_BWD_CASE(M, N)                                                              \
+  if (g.m == M && g.n == N)                                                             \
+    return bf16 ? launch_bwd_tma_io<IoBF16, M, N>(g, mx, mdy, dx, y, a, b, ws, grid, st) \
+                : launch_bwd_tma_io<IoF32, M, N>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+  GRK_TMA_DEGREES(GRK_BWD_CASE)
+#undef GRK_BWD_CASE
+  return cudaErrorNotSupported;
 }
 
 inline cudaError_t read_device_error(uint32_t* out, cudaStream_t st) {

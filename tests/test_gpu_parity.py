@@ -38,6 +38,16 @@ CASES = {
                        lo=-0.2, hi=0.2),
     "deg_5_0": _custom("deg_5_0", 60, 128, 8, 5, 0, synth.BF16),
     "deg_2_6": _custom("deg_2_6", 60, 96, 3, 2, 6, synth.F32),
+    # degrees with TMA-pipelined kernels besides (5, 4): several tiles and a ragged tail
+    "deg_3_3_bf16": _custom("deg_3_3", 530, 256, 4, 3, 3, synth.BF16),
+    "deg_4_4_f32": _custom("deg_4_4", 410, 256, 4, 4, 4, synth.F32),
+    "deg_5_5_bf16": _custom("deg_5_5", 530, 256, 4, 5, 5, synth.BF16),
+    "deg_6_6_f32": _custom("deg_6_6", 410, 256, 4, 6, 6, synth.F32, lo=-0.3, hi=0.3),
+    "deg_7_7_bf16": _custom("deg_7_7", 530, 256, 4, 7, 7, synth.BF16, lo=-0.3, hi=0.3),
+    "deg_8_8_bf16": _custom("deg_8_8b", 530, 256, 4, 8, 8, synth.BF16, lo=-0.2, hi=0.2),
+    # more groups than the kernels' shared coefficient table holds (64)
+    "ng96_bf16": _custom("ng96", 200, 3072, 96, 5, 4, synth.BF16),
+    "ng128_f32_deg66": _custom("ng128", 120, 3072, 128, 6, 6, synth.F32, lo=-0.3, hi=0.3),
 }
 
 _cache = {}
@@ -77,20 +87,23 @@ def test_forward_backward_parity(name, flags):
 
 def test_fast_path_is_taken_where_expected():
     for name in ("tiny", "kat_t_ragged", "kat_s_ragged", "kat_b_ragged", "stress_ng1",
-                 "stress_ng8", "stress_ng64", "one_row_bf16"):
+                 "stress_ng8", "stress_ng64", "one_row_bf16", "deg_8_8", "deg_3_3_bf16",
+                 "deg_4_4_f32", "deg_5_5_bf16", "deg_6_6_f32", "deg_7_7_bf16", "deg_8_8_bf16",
+                 "ng96_bf16", "ng128_f32_deg66"):
         w = CASES[name]
         t = torch.empty((w.rows, w.d), dtype=torch.float32 if w.dtype == synth.F32
                         else torch.bfloat16, device="cuda")
         args = (w.rows, 1, w.d, w.n_g, w.m, w.n, w.dtype)
         assert grk.grkan_forward_path(t, t, *args) == 1, name
         assert grk.grkan_backward_path(t, t, t, *args) == 1, name
-    for name in ("odd_f32_dg10", "odd_bf16_dg6", "deg_3_2", "deg_0_0", "deg_8_8"):
+    for name in ("odd_f32_dg10", "odd_bf16_dg6", "deg_3_2", "deg_0_0", "deg_5_0", "deg_2_6"):
         w = CASES[name]
         t = torch.empty((w.rows, w.d), dtype=torch.float32, device="cuda")
         assert grk.grkan_backward_path(t, t, t, w.rows, 1, w.d, w.n_g, w.m, w.n, w.dtype) == 0
 
 
-@pytest.mark.parametrize("name", ["kat_b_ragged", "stress_ng64", "kat_t_ragged", "odd_f32_dg10"])
+@pytest.mark.parametrize("name", ["kat_b_ragged", "stress_ng64", "kat_t_ragged", "odd_f32_dg10",
+                                  "ng96_bf16", "deg_7_7_bf16"])
 def test_bitwise_determinism(name):
     w, x, dy, a, b = case_data(name)[:5]
     tx, tdy, ta, tb = _dev(w, x, dy, a, b)
