@@ -19,6 +19,7 @@ __all__ = [
     "grkan_merge_ranks", "grkan_backward_noalloc", "NOALLOC_WORKSPACE_BYTES",
     "grkan_step_host", "grkan_step_host_scratch_bytes", "grkan_forward_backward",
     "grkan_backward_atomic", "ATOMIC_PER_ELEMENT", "ATOMIC_PER_BLOCK",
+    "grkan_linear_forward", "linear_forward",
     "forward_backward",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
     "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
@@ -67,6 +68,8 @@ def _load():
         "grkan_backward_merge": (S, [P, SZ, P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int,
                                      P]),
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
+        "grkan_linear_forward": (S, [P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I64,
+                                     ctypes.c_int, P]),
         "grkan_backward_atomic": (S, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                       ctypes.c_int, I32, I32, P]),
         "grkan_forward_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
@@ -178,6 +181,23 @@ def grkan_backward_noalloc(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, s
 
 ATOMIC_PER_ELEMENT = 1
 ATOMIC_PER_BLOCK = 2
+
+
+def grkan_linear_forward(x, a, b, W, bias, out, B, N, d, n_g, m, n, nout, dtype, stream=None):
+    return lib().grkan_linear_forward(_ptr(x), _ptr(a), _ptr(b), _ptr(W), _ptr(bias), _ptr(out),
+                                      B, N, d, n_g, m, n, nout, dtype, _stream(stream))
+
+
+def linear_forward(x, a, b, n_g, W, bias=None, stream=None):
+    """GR-KAN followed by a linear layer: (B, N, d) bf16 -> (B, N, nout) bf16."""
+    import torch
+    B, N, d, dt = _dims(x, n_g)
+    m, n = _coef(a, b, n_g)
+    nout = W.shape[0]
+    out = torch.empty(x.shape[:-1] + (nout,), dtype=x.dtype, device=x.device)
+    _check(grkan_linear_forward(x, a, b, W, bias, out, B, N, d, n_g, m, n, nout, dt, stream),
+           "grkan_linear_forward")
+    return out
 
 
 def grkan_backward_atomic(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, mode, block_rows=0,

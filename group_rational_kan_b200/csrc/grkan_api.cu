@@ -14,6 +14,7 @@
 #include "grkan_atomic.cuh"
 #include "grkan_common.cuh"
 #include "grkan_generic.cuh"
+#include "grkan_linear.cuh"
 #include "grkan_merge.cuh"
 #include "grkan_tma.cuh"
 
@@ -604,6 +605,75 @@ grkan_status_t grkan_backward_atomic(const void* x, const void* dy, const float*
               dA, dB, p.rows, p.d, (int)p.dg, p.n_g, p.m, p.n, sb);
   }
   return cuda_status(cudaGetLastError(), "grkan_backward_atomic launch");
+}
+
+namespace {
+
+bool make_map_sw128(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                    uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_last_error("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled not found", 0);
+    return false;
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t strides[1] = {(cuuint64_t)(inner * 2)};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) set_last_error("cuTensorMapEncodeTiled", "failed (linear)", (int)r);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* b, const void* W,
+                                    const float* bias, void* out, int64_t B, int64_t N,
+                                    int64_t d, int32_t n_g, int32_t m, int32_t n, int64_t nout,
+                                    grkan_dtype_t dtype, void* stream) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if (p.dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
+  if (p.m != 5 || p.n != 4) return GRKAN_ERR_DEGREE;
+  if (nout < 0 || p.d % grk::lin::BK != 0 || p.dg % 8 != 0 || nout % 8 != 0 ||
+      p.rows > 0x7fffffffLL || nout > 0x7fffffffLL)
+    return GRKAN_ERR_SHAPE;
+  if (p.rows == 0 || nout == 0) return GRKAN_OK;
+  if (!x || !W || !out) return GRKAN_ERR_NULL;
+  if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+  if (!aligned16(x) || !aligned16(W) || !aligned16(out)) return GRKAN_ERR_SHAPE;
+  const size_t xbytes = (size_t)p.rows * (size_t)p.d * 2;
+  const size_t wbytes = (size_t)nout * (size_t)p.d * 2;
+  const size_t obytes = (size_t)p.rows * (size_t)nout * 2;
+  if (overlaps(out, obytes, x, xbytes) || overlaps(out, obytes, W, wbytes)) return GRKAN_ERR_ALIAS;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  CUtensorMap mx, mw, mo;
+  if (!make_map_sw128(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, grk::lin::BK, grk::lin::BM) ||
+      !make_map_sw128(&mw, W, (uint64_t)p.d, (uint64_t)nout, grk::lin::BK, grk::lin::BN) ||
+      !make_map_sw128(&mo, out, (uint64_t)nout, (uint64_t)p.rows, grk::lin::kEpiCols,
+                      grk::lin::kEpiRows))
+    return GRKAN_ERR_CUDA;
+  grk::lin::LinGeom g;
+  g.rows = p.rows;
+  g.d = (int)p.d;
+  g.nout = (int)nout;
+  g.dg = (int)p.dg;
+  g.n_g = p.n_g;
+  g.kt = (int)(p.d / grk::lin::BK);
+  const long long tiles = ((p.rows + grk::lin::BM - 1) / grk::lin::BM) *
+                          ((nout + grk::lin::BN - 1) / grk::lin::BN);
+  if (tiles > 0x7fffffffLL) return GRKAN_ERR_SHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = grk::ensure_smem<grk::lin::linear_fwd>(grk::lin::Layout::kAlloc);
+  if (e == cudaSuccess) {
+    grk::lin::linear_fwd<<<(unsigned)tiles, grk::lin::kThreads, grk::lin::Layout::kAlloc, st>>>(
+        mx, mw, mo, a, b, bias, g);
+    e = cudaGetLastError();
+  }
+  return cuda_status(e, "grkan_linear_forward launch");
 }
 
 grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* dA, float* dB,

@@ -1,0 +1,348 @@
+// grkan_linear.cuh -- the GR-KAN activation fused into the linear layer that
+// follows it, on the fifth-generation tensor cores:
+//
+//   out[r, o] = sum_k y[r, k] W[o, k] (+ bias[o]),   y = P(x) / (1 + |Q(x)|)
+//
+// A KAT layer is a group-rational activation followed by a linear map
+// ("FlashKAT ...", paper notes, section "Insight 2": the GR-KAN term next to the
+// linear layer's 2 d_in d_out operations), and the pages locate what remains of
+// the training time after their fix in the GR-KAN forward. Here the activation
+// is computed while the tile of x waits in shared memory for the matrix
+// multiply, so y never goes to HBM.
+//
+// One CTA computes a 128 x 256 tile of out (bf16 in, float32 accumulate in
+// tensor memory, bf16 out), in K steps of 64:
+//   warp 0       lane 0 issues the TMA loads of the x tile (128 x 64) and the
+//                W tile (256 x 64), 128-byte swizzled, into a ring of stages;
+//   warps 2..9   apply the activation to the x tile in place (same swizzled
+//                positions), then signal the stage ready;
+//   warp 1       allocates 256 TMEM columns; lane 0 issues four
+//                tcgen05.mma (M 128, N 256, K 16) per stage and returns the
+//                stage to the producer with tcgen05.commit;
+//   warps 2..5   at the end read the accumulators (tcgen05.ld, one 32-lane
+//                quarter each), add the bias, convert to bf16 and write the
+//                tile through swizzled staging buffers with TMA stores.
+// Every wait is bounded (device error word, as in the other kernels); TMEM is
+// freed on every path.
+#pragma once
+
+#include "grkan_tma.cuh"
+
+namespace grk {
+namespace lin {
+
+constexpr int BM = 128;  // rows of a tile (UMMA M)
+constexpr int BN = 256;  // output features of a tile (UMMA N)
+constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
+constexpr int kStages = 4;
+constexpr int kXformWarps = 8;
+constexpr int kWarps = 2 + kXformWarps;
+constexpr int kThreads = kWarps * 32;
+constexpr unsigned kATile = BM * BK * 2;  // 16 KiB
+constexpr unsigned kBTile = BN * BK * 2;  // 32 KiB
+constexpr unsigned kStage = kATile + kBTile;
+constexpr unsigned kEpiRows = 32;         // rows per epilogue warp
+constexpr unsigned kEpiCols = 64;         // columns per TMA store box (128 bytes of bf16)
+constexpr unsigned kEpiBuf = kEpiRows * kEpiCols * 2;  // 4 KiB staging buffer
+
+// Shared memory: [stages][A | B] at a 1024-byte boundary, then the barriers
+// (full, ready, empty per stage; accumulator full), the TMEM address slot and
+// the coefficient table.
+struct Layout {
+  static constexpr unsigned kBarOff = kStages * kStage;
+  static constexpr unsigned kNumBars = 3 * kStages + 1;
+  static constexpr unsigned kTmemSlot = kBarOff + kNumBars * 8;
+  static constexpr unsigned kTabOff = (kTmemSlot + 4 + 15) / 16 * 16;
+  static constexpr unsigned kBytes = kTabOff + coef_table_bytes<5, 4>();
+  static constexpr unsigned kAlloc = kBytes + 1024;  // slack to align the base to 1024
+};
+
+// --- tcgen05 wrappers ---------------------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem] B[smem]^T, kind::f16 (bf16 inputs, float32 accumulator)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on an mbarrier once every tcgen05 operation issued so far by this thread is done
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// 16 consecutive float32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
+// 128-byte swizzling: rows of 128 bytes, 8-row atoms of 1024 bytes one after
+// another (stride byte offset 1024), descriptor version 1, layout SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor: float32 accumulator, bf16 A and B, both K-major,
+// N = BN, M = BM.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+struct LinGeom {
+  long long rows;  // R = B * N
+  int d;           // K: input features (the activation's channels)
+  int nout;        // output features
+  int dg;          // channels per group
+  int n_g;
+  int kt;          // K steps = d / BK
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mw,
+           const __grid_constant__ CUtensorMap mo, const float* __restrict__ a,
+           const float* __restrict__ b, const float* __restrict__ bias, const LinGeom geom) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + Layout::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+  auto ready_bar = [&](int s) { return bar0 + 8u * (uint32_t)(kStages + s); };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * kStages + s); };
+  const uint32_t acc_bar = bar0 + 8u * (uint32_t)(3 * kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Layout::kTmemSlot);
+  float* ctab = reinterpret_cast<float*>(smem + Layout::kTabOff);
+  const bool use_tab = geom.n_g <= kTableGroups;
+
+  const int n_tiles = (geom.nout + BN - 1) / BN;
+  const int n0 = (int)(blockIdx.x % n_tiles) * BN;
+  const long long m0 = (long long)(blockIdx.x / n_tiles) * BM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(ready_bar(s), kXformWarps);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+    prefetch_map(&mx);
+    prefetch_map(&mw);
+    prefetch_map(&mo);
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + Layout::kTmemSlot, (uint32_t)BN);
+    tmem_relinquish();
+  }
+  if (use_tab) build_coef_table<5, 4>(ctab, a, b, geom.n_g);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---- TMA producer -------------------------------------------------------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int kt = 0; kt < geom.kt; ++kt) {
+        const int s = kt % kStages;
+        if (kt >= kStages &&
+            !mbar_wait(empty_bar(s), (uint32_t)((kt / kStages) - 1) & 1u)) {
+          report(kErrEmptyWait);
+          ok = false;
+          break;
+        }
+        const uint32_t sa = sbase + (uint32_t)s * kStage;
+        mbar_arrive_expect_tx(full_bar(s), kStage);
+        tma_load_2d(sa, &mx, kt * BK, (int)m0, full_bar(s));
+        tma_load_2d(sa + kATile, &mw, kt * BK, n0, full_bar(s));
+        ++issued;
+      }
+      if (!ok) {  // let the issued loads land before the CTA's memory goes away
+        for (int j = 0; j < issued; ++j)
+          if (!mbar_wait(full_bar(j % kStages), (uint32_t)(j / kStages) & 1u)) report(kErrDrainWait);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issue ----------------------------------------------------------------
+    if (lane == 0) {
+      for (int kt = 0; kt < geom.kt; ++kt) {
+        const int s = kt % kStages;
+        const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+        if (!mbar_wait(full_bar(s), ph) || !mbar_wait(ready_bar(s), ph)) {
+          report(kErrFullWait);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = sbase + (uint32_t)s * kStage;
+        const uint64_t ad = sw128_desc(sa);
+        const uint64_t bd = sw128_desc(sa + kATile);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes = 2 descriptor units per step
+          umma_bf16(tmem_d, ad + 2u * (uint64_t)k, bd + 2u * (uint64_t)k, kIdesc,
+                    (kt > 0 || k > 0) ? 1u : 0u);
+        umma_commit(empty_bar(s));
+      }
+      umma_commit(acc_bar);  // every MMA issued above is done when this arrives
+      // and none may still write TMEM when the columns are freed
+      if (!mbar_wait(acc_bar, 0)) report(kErrReduceWait);
+    }
+  } else {
+    // ---- activation in place, then the epilogue -----------------------------------
+    const int t = threadIdx.x - 64;  // 0..255
+    const int j = t & 7;             // logical 16-byte chunk (8 channels) of a 128-byte row
+    const int rb = t >> 3;           // rows rb, rb + 32, rb + 64, rb + 96
+    Coef54 c;
+    int cur_g = -1;
+    for (int kt = 0; kt < geom.kt; ++kt) {
+      const int s = kt % kStages;
+      const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+      if (!mbar_wait(full_bar(s), ph)) {
+        report(kErrFullWait);
+        ok = false;
+        break;
+      }
+      const int g = (kt * BK + j * 8) / geom.dg;
+      if (g != cur_g) {
+        load_coef<5, 4>(use_tab, ctab, a, b, g, c);
+        cur_g = g;
+      }
+      unsigned char* at = smem + (size_t)s * kStage;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = rb + 32 * i;
+        uint4* p = reinterpret_cast<uint4*>(at + r * 128 + ((j ^ (r & 7)) << 4));
+        uint4 v = *p;
+        v.x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.x)));
+        v.y = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.y)));
+        v.z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.z)));
+        v.w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.w)));
+        *p = v;
+      }
+      fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ready_bar(s));
+    }
+    // epilogue: warps 2..5, TMEM lane quarter = warp % 4
+    if (warp < 6) {
+      const int q = warp & 3;
+      if (!mbar_wait(acc_bar, 0)) {
+        report(kErrReduceWait);
+        ok = false;
+      }
+      tc_fence_after();
+      if (ok) {
+        // staging buffer of this warp inside the (now idle) stage ring, 1024-aligned
+        unsigned char* stg = smem + (size_t)(warp - 2) * 2 * kEpiBuf;
+        const uint32_t stg_a = sbase + (uint32_t)(warp - 2) * 2u * kEpiBuf;
+        for (int cb = 0; cb < BN / (int)kEpiCols; ++cb) {
+          const int col0 = n0 + cb * (int)kEpiCols;
+          if (col0 >= geom.nout) break;
+          const int buf = cb & 1;
+          if (cb >= 2) {  // the store that used this buffer has read it
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+          }
+          unsigned char* sb = stg + buf * kEpiBuf;
+#pragma unroll
+          for (int h = 0; h < (int)kEpiCols / 16; ++h) {
+            float v[16];
+            tmem_ld16(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(cb * kEpiCols + h * 16), v);
+            if (bias) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int col = col0 + h * 16 + e;
+                v[e] += col < geom.nout ? __ldg(bias + col) : 0.f;
+              }
+            }
+            // two 16-byte chunks (logical 2h, 2h + 1) of this row, swizzled
+            uint4 w0, w1;
+            w0.x = f2_to_bf16x2(make_float2(v[0], v[1]));
+            w0.y = f2_to_bf16x2(make_float2(v[2], v[3]));
+            w0.z = f2_to_bf16x2(make_float2(v[4], v[5]));
+            w0.w = f2_to_bf16x2(make_float2(v[6], v[7]));
+            w1.x = f2_to_bf16x2(make_float2(v[8], v[9]));
+            w1.y = f2_to_bf16x2(make_float2(v[10], v[11]));
+            w1.z = f2_to_bf16x2(make_float2(v[12], v[13]));
+            w1.w = f2_to_bf16x2(make_float2(v[14], v[15]));
+            *reinterpret_cast<uint4*>(sb + lane * 128 + (((2 * h) ^ (lane & 7)) << 4)) = w0;
+            *reinterpret_cast<uint4*>(sb + lane * 128 + (((2 * h + 1) ^ (lane & 7)) << 4)) = w1;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&mo, stg_a + (uint32_t)buf * kEpiBuf, col0, (int)m0 + q * 32);
+            bulk_commit();
+          }
+        }
+        if (lane == 0) bulk_wait0();
+        __syncwarp();
+      }
+    }
+  }
+  // teardown: every tcgen05.ld has completed; free the accumulator columns
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, (uint32_t)BN);
+  }
+}
+
+}  // namespace lin
+}  // namespace grk

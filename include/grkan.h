@@ -130,6 +130,24 @@ GRKAN_API grkan_status_t grkan_forward_backward(const void* x, const void* dy, c
                                                 size_t workspace_bytes, uint32_t flags,
                                                 void* stream);
 
+/* The GR-KAN activation fused into the linear layer that follows it (a KAT
+ * layer: "FlashKAT: Understanding and Addressing Performance Bottlenecks in the
+ * Kolmogorov-Arnold Transformer", paper notes, section "Insight 2"):
+ *   out[r, o] = sum_k y[r, k] W[o, k] + bias[o],   y = grkan_forward(x),
+ * on the tensor cores, with y computed in shared memory and never written.
+ * x: bf16 (B*N rows x d), row-major. W: bf16 (nout x d), row-major (a linear
+ * layer's weight). bias: float32 (nout) or NULL. out: bf16 (B*N x nout),
+ * row-major, overwritten. y is rounded to bf16 before the product, as when
+ * grkan_forward's output feeds a bf16 matrix multiply; the sum is float32.
+ * Requires dtype GRKAN_BF16 (else GRKAN_ERR_DTYPE), (m, n) = (5, 4) (else
+ * GRKAN_ERR_DEGREE), d % 64 == 0, d_g % 8 == 0, nout % 8 == 0 and 16-byte
+ * aligned x, W, out (else GRKAN_ERR_SHAPE); out may not overlap x or W. */
+GRKAN_API grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* b,
+                                              const void* W, const float* bias, void* out,
+                                              int64_t B, int64_t N, int64_t d, int32_t n_g,
+                                              int32_t m, int32_t n, int64_t nout,
+                                              grkan_dtype_t dtype, void* stream);
+
 /* Coefficient gradients accumulated with float32 atomic adds, the two schemes
  * that "FlashKAT: Understanding and Addressing Performance Bottlenecks in the
  * Kolmogorov-Arnold Transformer" compares (paper notes, sections "2. The

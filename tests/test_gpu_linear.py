@@ -1,0 +1,88 @@
+"""GR-KAN fused into the following linear layer (grkan_linear_forward) against
+the fp64 oracle's activation times the weight in fp64, and against the same
+product taken from the library's own forward output. Shapes span several
+128-row and 256-column tiles, a ragged last tile in both, more K steps than the
+kernel's four-stage ring, groups that straddle a 64-channel K step, bias and no
+bias."""
+import numpy as np
+import pytest
+import torch
+
+import group_rational_kan_b200 as grk
+import oracle
+import synth
+from parity import to_f64, to_torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(rows, d, n_g, nout, seed=0, dy_scale=1.0):
+    w = synth.Workload(name="lin", B=rows, N=1, d=d, n_g=n_g, m=5, n=4, dtype=synth.BF16,
+                       x_kind=synth.KIND_NORMAL, x_scale=1.0, x_clip=8.0, dy_scale=dy_scale,
+                       coef_base="zero", coef_lo=-0.5, coef_hi=0.5, seed=seed)
+    x = w.x()
+    a, b = w.coefficients()
+    # the weight: seeded bf16 from the same generator (the dy stream, scaled)
+    wt = synth.Workload(name="lin_w", B=nout, N=1, d=d, n_g=n_g, m=5, n=4, dtype=synth.BF16,
+                        x_kind=synth.KIND_NORMAL, x_scale=1.0, x_clip=8.0,
+                        dy_scale=1.0 / np.sqrt(d), coef_base="zero", coef_lo=-0.5,
+                        coef_hi=0.5, seed=seed + 1).dy()
+    bias = np.linspace(-0.25, 0.25, nout).astype(np.float32)
+    return w, x, a, b, wt, bias
+
+
+def _reference(w, x, a, b, wt, bias):
+    y = oracle.forward(x, a, b, w.n_g)  # fp64
+    W = synth.bf16_bits_to_f32(wt).astype(np.float64)
+    ref = y @ W.T
+    scale = np.abs(y) @ np.abs(W).T
+    if bias is not None:
+        ref = ref + bias.astype(np.float64)[None, :]
+    return ref, scale
+
+
+@pytest.mark.parametrize("rows,d,n_g,nout,with_bias", [
+    (300, 768, 8, 576, True),     # d_g 96: K steps straddle groups; ragged rows and columns
+    (128, 256, 4, 256, False),    # one tile exactly
+    (1000, 3072, 8, 768, True),   # the KAT-B second-linear shape, ragged rows
+])
+def test_fused_linear_matches_oracle(rows, d, n_g, nout, with_bias):
+    w, x, a, b, wt, bias = _case(rows, d, n_g, nout)
+    tx = to_torch(x)
+    tw = to_torch(wt)
+    ta = torch.from_numpy(a).cuda()
+    tb = torch.from_numpy(b).cuda()
+    tbias = torch.from_numpy(bias).cuda() if with_bias else None
+    out = grk.linear_forward(tx, ta, tb, n_g, tw, tbias)
+    torch.cuda.synchronize()
+    assert grk.grkan_device_error()[1] == 0
+    got = to_f64(out)
+    ref, scale = _reference(w, x, a, b, wt, bias if with_bias else None)
+    # y rounded to bf16 (2^-9 relative per term), float32 sums, bf16 output (2^-9)
+    lim = 2.0 ** -8 * scale + 2.0 ** -8 * np.abs(ref) + 1e-6
+    err = np.abs(got - ref)
+    assert np.all(err <= lim), "worst %.3g of limit" % float(np.max(err / lim))
+
+    # the unfused composition: the library's forward (same y bits), then the
+    # product in float32 on the device
+    y = grk.forward(tx, ta, tb, n_g)
+    ref2 = y.float() @ tw.float().T
+    if with_bias:
+        ref2 += tbias
+    ref2 = ref2.double().cpu().numpy()
+    err2 = np.abs(got - ref2)
+    lim2 = 2.0 ** -8 * np.abs(ref2) + 1e-5 * scale + 1e-6
+    assert np.all(err2 <= lim2), "worst %.3g of limit" % float(np.max(err2 / lim2))
+
+
+def test_fused_linear_rejects_unsupported():
+    t = torch.empty(64, dtype=torch.bfloat16, device="cuda")
+    f = torch.empty(16, device="cuda")
+    args = (1, 1, 64, 8, 5, 4, 64)
+    assert grk.grkan_linear_forward(t, f, f, t, None, t, *args, grk.F32) == 4  # dtype
+    assert grk.grkan_linear_forward(t, f, f, t, None, t, 1, 1, 64, 8, 3, 3, 64,
+                                    grk.BF16) == 3  # degree
+    assert grk.grkan_linear_forward(t, f, f, t, None, t, 1, 1, 96, 8, 5, 4, 64,
+                                    grk.BF16) == 2  # d % 64
+    assert grk.grkan_linear_forward(t, f, f, t, None, t, 0, 1, 64, 8, 5, 4, 64,
+                                    grk.BF16) == 0  # empty: nothing to do
