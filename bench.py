@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused-launches", type=int, default=50,
                     help="launches of the recompute variant timed after the step (0: skip)")
+    ap.add_argument("--linear-nout", type=int, default=0,
+                    help="also time the activation fused into a following linear layer with "
+                         "this many outputs (bf16 workloads; 0: skip)")
     return ap.parse_args()
 
 
@@ -329,6 +332,43 @@ def main():
         torch.cuda.synchronize(dev)
         fused_ms = f0.elapsed_time(f1) / args.fused_launches
 
+    # the activation fused into a following linear layer (bf16 only), outside the
+    # timed step: fused kernel against the activation kernel plus cuBLAS
+    linear = None
+    if args.linear_nout > 0 and dt == synth.BF16 and (m, n) == (5, 4):
+        nout = args.linear_nout
+        gen = torch.Generator(device=dev).manual_seed(1234 + rank)
+        Wl = (torch.randn(nout, d, device=dev, generator=gen) / d ** 0.5).to(torch.bfloat16)
+        outl = torch.empty((B * N, nout), dtype=torch.bfloat16, device=dev)
+
+        def lin_fused():
+            check(grk.grkan_linear_forward(x, a, b, Wl, None, outl, B, N, d, n_g, m, n, nout, dt,
+                                           sp), "linear_forward")
+
+        def lin_unfused():
+            check(grk.grkan_forward(x, y, a, b, B, N, d, n_g, m, n, dt, sp), "forward")
+            torch.matmul(y.view(B * N, d), Wl.t(), out=outl)
+
+        def timed(f, k=20):
+            for _ in range(3):
+                f()
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(k):
+                f()
+            t1.record(stream)
+            torch.cuda.synchronize(dev)
+            return t0.elapsed_time(t1) / k
+
+        fl = 2.0 * B * N * d * nout
+        f_ms, u_ms = timed(lin_fused), timed(lin_unfused)
+        linear = {"nout": nout, "fused_ms": f_ms, "unfused_ms": u_ms,
+                  "fused_TFLOP/s": fl / (f_ms * 1e-3) / 1e12,
+                  "note": "grkan_linear_forward vs grkan_forward + torch.matmul (cuBLAS), "
+                          "no bias; not part of the timed step"}
+        del Wl, outl
+
     # end to end through the C ABI's host-buffer entry point: pinned inputs in,
     # y, dx and dA/dB out, copies inside the timed region (chunks streamed over
     # three streams so that copies in, kernels and copies out overlap)
@@ -410,6 +450,7 @@ def main():
                 "h2d_bytes_per_step": 2 * nbytes,
                 "d2h_bytes_per_step": 2 * nbytes + (n_g * K) * 4, "ms_per_step": e2e_ms,
                 "api": "grkan_step_host (x, dy in; y, dx, dA, dB out; pinned host buffers)"},
+        "fused_linear": linear,
         "gpu_launches": args.steps * (3 + (1 if world > 1 else 0)),
         "clocks": clocks,
         "device_error": derr,
