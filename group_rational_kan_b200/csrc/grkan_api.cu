@@ -609,8 +609,10 @@ grkan_status_t grkan_backward_atomic(const void* x, const void* dy, const float*
 
 namespace {
 
-bool make_map_sw128(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                    uint32_t box_inner, uint32_t box_outer) {
+// 2-D bf16 tensor map with the given shared-memory swizzle (the inner box must
+// span no more bytes than the swizzle width).
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_last_error("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled not found", 0);
@@ -621,7 +623,7 @@ bool make_map_sw128(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) set_last_error("cuTensorMapEncodeTiled", "failed (linear)", (int)r);
   return r == CUDA_SUCCESS;
@@ -651,10 +653,12 @@ grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* 
   if (overlaps(out, obytes, x, xbytes) || overlaps(out, obytes, W, wbytes)) return GRKAN_ERR_ALIAS;
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
   CUtensorMap mx, mw, mo;
-  if (!make_map_sw128(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, grk::lin::BK, grk::lin::BM) ||
-      !make_map_sw128(&mw, W, (uint64_t)p.d, (uint64_t)nout, grk::lin::BK, grk::lin::BN) ||
-      !make_map_sw128(&mo, out, (uint64_t)nout, (uint64_t)p.rows, grk::lin::kEpiCols,
-                      grk::lin::kEpiRows))
+  if (!make_map_bf16(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, grk::lin::BK, grk::lin::BM,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_bf16(&mw, W, (uint64_t)p.d, (uint64_t)nout, grk::lin::BK, grk::lin::BNH,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_bf16(&mo, out, (uint64_t)nout, (uint64_t)p.rows, grk::lin::kEpiCols,
+                     grk::lin::kEpiRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return GRKAN_ERR_CUDA;
   grk::lin::LinGeom g;
   g.rows = p.rows;

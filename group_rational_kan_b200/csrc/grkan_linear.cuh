@@ -10,18 +10,23 @@
 // is computed while the tile of x waits in shared memory for the matrix
 // multiply, so y never goes to HBM.
 //
-// One CTA computes a 128 x 256 tile of out (bf16 in, float32 accumulate in
-// tensor memory, bf16 out), in K steps of 64:
-//   warp 0       lane 0 issues the TMA loads of the x tile (128 x 64) and the
-//                W tile (256 x 64), 128-byte swizzled, into a ring of stages;
-//   warps 2..9   apply the activation to the x tile in place (same swizzled
+// One CTA computes a 128 x 512 tile of out (bf16 in, float32 accumulate in all
+// 512 TMEM columns, bf16 out), in K steps of 32, so that the activation of an x
+// tile serves 512 output features:
+//   warp 0       lane 0 issues the TMA loads of the x tile (128 x 32) and of
+//                the W tile (two 256 x 32 halves), 64-byte swizzled, into a
+//                ring of stages;
+//   warps 2..17  apply the activation to the x tile in place (same swizzled
 //                positions), then signal the stage ready;
-//   warp 1       allocates 256 TMEM columns; lane 0 issues four
-//                tcgen05.mma (M 128, N 256, K 16) per stage and returns the
-//                stage to the producer with tcgen05.commit;
+//   warp 1       allocates the TMEM columns; lane 0 issues two tcgen05.mma
+//                (M 128, N 256, K 16) per half and stage and returns the stage
+//                to the producer with tcgen05.commit;
 //   warps 2..5   at the end read the accumulators (tcgen05.ld, one 32-lane
 //                quarter each), add the bias, convert to bf16 and write the
-//                tile through swizzled staging buffers with TMA stores.
+//                tile through 128-byte-swizzled staging buffers with TMA
+//                stores.
+// A tile whose second half lies past n_out issues neither its loads nor its
+// MMAs.
 // Every wait is bounded (device error word, as in the other kernels); TMEM is
 // freed on every path.
 #pragma once
@@ -31,15 +36,22 @@
 namespace grk {
 namespace lin {
 
-constexpr int BM = 128;  // rows of a tile (UMMA M)
-constexpr int BN = 256;  // output features of a tile (UMMA N)
-constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 4;
-constexpr int kXformWarps = 8;
+constexpr int BM = 128;   // rows of a tile (UMMA M)
+constexpr int BNH = 256;  // output features of one MMA (UMMA N), a tile half
+constexpr int BN = 2 * BNH;
+constexpr int BK = 32;    // K per stage: one 64-byte swizzle row of bf16
+constexpr int kStages = 5;
+#ifndef GRK_LIN_XFORM_WARPS
+#define GRK_LIN_XFORM_WARPS 16
+#endif
+constexpr int kXformWarps = GRK_LIN_XFORM_WARPS;  // warps applying the activation
+constexpr int kChunksPerRow = BK * 2 / 16;                        // 16-byte chunks per row
+constexpr int kXformRows = BM * kChunksPerRow / (kXformWarps * 32);  // rows per transform thread
 constexpr int kWarps = 2 + kXformWarps;
 constexpr int kThreads = kWarps * 32;
-constexpr unsigned kATile = BM * BK * 2;  // 16 KiB
-constexpr unsigned kBTile = BN * BK * 2;  // 32 KiB
+constexpr unsigned kATile = BM * BK * 2;    // 8 KiB
+constexpr unsigned kBHalf = BNH * BK * 2;   // 16 KiB
+constexpr unsigned kBTile = 2 * kBHalf;     // 32 KiB
 constexpr unsigned kStage = kATile + kBTile;
 constexpr unsigned kEpiRows = 32;         // rows per epilogue warp
 constexpr unsigned kEpiCols = 64;         // columns per TMA store box (128 bytes of bf16)
@@ -126,16 +138,16 @@ __device__ __forceinline__ void bulk_wait0() {
 }
 
 // Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
-// 128-byte swizzling: rows of 128 bytes, 8-row atoms of 1024 bytes one after
-// another (stride byte offset 1024), descriptor version 1, layout SWIZZLE_128B.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
-         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+// 64-byte swizzling: rows of 64 bytes, 8-row atoms of 512 bytes one after
+// another (stride byte offset 512), descriptor version 1, layout SWIZZLE_64B.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(512u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)4u << 61);
 }
 
 // Instruction descriptor: float32 accumulator, bf16 A and B, both K-major,
-// N = BN, M = BM.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+// N = BNH, M = BM.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BNH >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
 struct LinGeom {
@@ -169,6 +181,7 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
   const int n_tiles = (geom.nout + BN - 1) / BN;
   const int n0 = (int)(blockIdx.x % n_tiles) * BN;
   const long long m0 = (long long)(blockIdx.x / n_tiles) * BM;
+  const bool two = n0 + BNH < geom.nout;  // the tile's second half holds outputs
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -184,7 +197,7 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
     prefetch_map(&mo);
   }
   if (warp == 1) {
-    tmem_alloc(sbase + Layout::kTmemSlot, (uint32_t)BN);
+    tmem_alloc(sbase + Layout::kTmemSlot, (uint32_t)BN);  // 512 columns: both halves
     tmem_relinquish();
   }
   if (use_tab) build_coef_table<5, 4>(ctab, a, b, geom.n_g);
@@ -207,9 +220,10 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
           break;
         }
         const uint32_t sa = sbase + (uint32_t)s * kStage;
-        mbar_arrive_expect_tx(full_bar(s), kStage);
+        mbar_arrive_expect_tx(full_bar(s), two ? kStage : kATile + kBHalf);
         tma_load_2d(sa, &mx, kt * BK, (int)m0, full_bar(s));
         tma_load_2d(sa + kATile, &mw, kt * BK, n0, full_bar(s));
+        if (two) tma_load_2d(sa + kATile + kBHalf, &mw, kt * BK, n0 + BNH, full_bar(s));
         ++issued;
       }
       if (!ok) {  // let the issued loads land before the CTA's memory goes away
@@ -230,12 +244,16 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
         }
         tc_fence_after();
         const uint32_t sa = sbase + (uint32_t)s * kStage;
-        const uint64_t ad = sw128_desc(sa);
-        const uint64_t bd = sw128_desc(sa + kATile);
+        const uint64_t ad = sw64_desc(sa);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes = 2 descriptor units per step
-          umma_bf16(tmem_d, ad + 2u * (uint64_t)k, bd + 2u * (uint64_t)k, kIdesc,
-                    (kt > 0 || k > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !two) break;
+          const uint64_t bd = sw64_desc(sa + kATile + (uint32_t)h * kBHalf);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes = 2 descriptor units per step
+            umma_bf16(tmem_d + (uint32_t)(h * BNH), ad + 2u * (uint64_t)k, bd + 2u * (uint64_t)k,
+                      kIdesc, (kt > 0 || k > 0) ? 1u : 0u);
+        }
         umma_commit(empty_bar(s));
       }
       umma_commit(acc_bar);  // every MMA issued above is done when this arrives
@@ -244,9 +262,10 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
     }
   } else {
     // ---- activation in place, then the epilogue -----------------------------------
-    const int t = threadIdx.x - 64;  // 0..255
-    const int j = t & 7;             // logical 16-byte chunk (8 channels) of a 128-byte row
-    const int rb = t >> 3;           // rows rb, rb + 32, rb + 64, rb + 96
+    const int t = threadIdx.x - 64;      // 0 .. 32 kXformWarps - 1
+    const int j = t % kChunksPerRow;     // logical 16-byte chunk (8 channels) of a row
+    const int rb = t / kChunksPerRow;    // rows rb + i kRowStep, i < kXformRows
+    constexpr int kRowStep = kXformWarps * 32 / kChunksPerRow;
     Coef54 c;
     int cur_g = -1;
     for (int kt = 0; kt < geom.kt; ++kt) {
@@ -257,23 +276,32 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
         ok = false;
         break;
       }
-      const int g = (kt * BK + j * 8) / geom.dg;
+      const int g = (kt * BK + j * 8) / geom.dg;  // a chunk lies in one group (d_g % 8 == 0)
       if (g != cur_g) {
         load_coef<5, 4>(use_tab, ctab, a, b, g, c);
         cur_g = g;
       }
       unsigned char* at = smem + (size_t)s * kStage;
+      // all loads first, then the arithmetic, then all stores: independent chunks
+      // in flight together
+      uint4* p[kXformRows];
+      uint4 v[kXformRows];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = rb + 32 * i;
-        uint4* p = reinterpret_cast<uint4*>(at + r * 128 + ((j ^ (r & 7)) << 4));
-        uint4 v = *p;
-        v.x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.x)));
-        v.y = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.y)));
-        v.z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.z)));
-        v.w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.w)));
-        *p = v;
+      for (int i = 0; i < kXformRows; ++i) {
+        const int r = rb + kRowStep * i;
+        // 64-byte swizzle: chunk bits [4, 6) of the offset xor row bits [1, 3)
+        p[i] = reinterpret_cast<uint4*>(at + r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+        v[i] = *p[i];
       }
+#pragma unroll
+      for (int i = 0; i < kXformRows; ++i) {
+        v[i].x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[i].x)));
+        v[i].y = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[i].y)));
+        v[i].z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[i].z)));
+        v[i].w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v[i].w)));
+      }
+#pragma unroll
+      for (int i = 0; i < kXformRows; ++i) *p[i] = v[i];
       fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
       __syncwarp();
       if (lane == 0) mbar_arrive(ready_bar(s));

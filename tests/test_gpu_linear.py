@@ -42,9 +42,12 @@ def _reference(w, x, a, b, wt, bias):
 
 
 @pytest.mark.parametrize("rows,d,n_g,nout,with_bias", [
-    (300, 768, 8, 576, True),     # d_g 96: K steps straddle groups; ragged rows and columns
-    (128, 256, 4, 256, False),    # one tile exactly
+    (300, 768, 8, 576, True),     # d_g 96: ragged rows and columns; second tile half-empty
+    (128, 256, 4, 256, False),    # one tile, first half only
+    (256, 512, 4, 1024, True),    # two full 512-column tiles
     (1000, 3072, 8, 768, True),   # the KAT-B second-linear shape, ragged rows
+    (200, 1536, 16, 200, False),  # n_out not a multiple of 64: the store box is clipped
+    (130, 160, 20, 520, True),    # d_g 8 (many groups per K step), n_out just past a tile
 ])
 def test_fused_linear_matches_oracle(rows, d, n_g, nout, with_bias):
     w, x, a, b, wt, bias = _case(rows, d, n_g, nout)
@@ -82,7 +85,7 @@ def test_fused_linear_rejects_unsupported():
     assert grk.grkan_linear_forward(t, f, f, t, None, t, *args, grk.F32) == 4  # dtype
     assert grk.grkan_linear_forward(t, f, f, t, None, t, 1, 1, 64, 8, 3, 3, 64,
                                     grk.BF16) == 3  # degree
-    assert grk.grkan_linear_forward(t, f, f, t, None, t, 1, 1, 96, 8, 5, 4, 64,
-                                    grk.BF16) == 2  # d % 64
+    assert grk.grkan_linear_forward(t, f, f, t, None, t, 1, 1, 48, 6, 5, 4, 64,
+                                    grk.BF16) == 2  # d % 32
     assert grk.grkan_linear_forward(t, f, f, t, None, t, 0, 1, 64, 8, 5, 4, 64,
                                     grk.BF16) == 0  # empty: nothing to do
