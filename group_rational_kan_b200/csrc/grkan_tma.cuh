@@ -21,6 +21,8 @@
 // g_grkan_device_error and the kernel winds down instead of hanging.
 #pragma once
 
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -970,17 +972,18 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
 // on the kernel itself).
 template <auto Kernel>
 inline cudaError_t ensure_smem(unsigned bytes) {
-  static int done_for_device = -1;
+  static std::atomic<unsigned long long> done_devices{0};  // bit d: set on device d
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (done_for_device == dev) return cudaSuccess;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done_devices.load(std::memory_order_acquire) & bit)) return cudaSuccess;
   const void* fn = reinterpret_cast<const void*>(Kernel);
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess) done_for_device = dev;
+  if (e == cudaSuccess && bit) done_devices.fetch_or(bit, std::memory_order_release);
   return e;
 }
 
