@@ -416,6 +416,11 @@ def main():
     step_bytes = accounting.bytes_per_element("step", dt) * E
     fused_bytes = accounting.bytes_per_element("forward_backward", dt) * E
     achieved = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    clk = clocks or {}
+    clk_mhz = float(clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0)
+    alu_ops = accounting.backward_fma_ops_per_element(m, n) * E
+    alu_peak = accounting.fma_pipe_peak(sms, clk_mhz)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -433,6 +438,15 @@ def main():
                                      "elements (profiles/bwd_tma_kat_b.md)",
                      "peak_source": peak_src,
                      "bytes_per_launch": bwd_bytes, "launch_ms": bwd_ms},
+        # the backward kernel is bound by FP32 arithmetic, not HBM: the same
+        # launch against the FMA pipe's peak at the median SM clock seen under load
+        "roofline_alu": {
+            "bound": "alu", "kernel": "backward stage 1 (dx + dA/dB partials)",
+            "achieved": alu_ops / (bwd_ms * 1e-3) / 1e9, "peak": alu_peak / 1e9,
+            "unit": "Gop/s", "frac": alu_ops / (bwd_ms * 1e-3) / alu_peak,
+            "ops_per_element": accounting.backward_fma_ops_per_element(m, n),
+            "peak_source": "128 FMA-pipe lane operations per SM-cycle x %d SMs x %.0f MHz "
+                           "(median SM clock during the timed region)" % (sms, clk_mhz)},
         "kernels": {
             "forward": {"ms": fwd_ms, "GB/s": fwd_bytes / (fwd_ms * 1e-3) / 1e9,
                         "frac": fwd_bytes / (fwd_ms * 1e-3) / 1e9 / peak},

@@ -46,3 +46,20 @@ def flashkat_access_reduction(s_block, d_g):
     the global accesses for the gradient (section "3. FlashKAT kernel
     restructuring (Algorithm 2)")."""
     return s_block * d_g
+
+
+def backward_fma_ops_per_element(m, n):
+    """FP32 FMA-pipe lane operations per element of the backward kernel (a packed
+    f32x2 operation counts two, one per element): powers x^2..x^k (k = max(m, n),
+    k - 1), P (m), P' (m - 1), Q (n), Q' (n - 1), y, t, -t y s (3), dx (2), the
+    m + 1 + n sums, and the scalar 1 + |Q|: k + 3m + 3n + 4. For (5, 4) that is 36,
+    which the instruction-class counters of the (5, 4) kernel confirm (25 FFMA2 +
+    9 FMUL2 + 1 FADD2 per element pair, plus 2 FADD)."""
+    return max(m, n) + 3 * m + 3 * n + 4
+
+
+def fma_pipe_peak(sms, sm_mhz):
+    """FP32 FMA-pipe lane operations per second: 128 per SM and cycle (a packed
+    f32x2 instruction issues 64 lane operations and holds the pipe two cycles)."""
+    return 128.0 * sms * sm_mhz * 1e6
+
