@@ -255,6 +255,8 @@ def test_fused_recompute_parity(name, flags):
     check_dx(to_f64(dx), dx_ref, ex, rtol, "%s fused dx" % name)
     check_coef(dA.cpu().numpy(), dB.cpu().numpy(), g_ref, what=name)
     assert torch.equal(dx, sdx) and torch.equal(dA, sdA) and torch.equal(dB, sdB)
+    # the recomputed y is the forward's, bit for bit
+    assert torch.equal(y, grk.forward(tx, ta, tb, w.n_g, flags=flags))
     assert grk.grkan_device_error()[1] == 0
 
 
