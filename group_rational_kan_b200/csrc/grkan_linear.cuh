@@ -146,9 +146,11 @@ __device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: float32 accumulator, bf16 A and B, both K-major,
-// N = BNH, M = BM.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BNH >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// M = BM, and N (a multiple of 16 up to BNH) in bits [17, 23) as N / 8.
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BM >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_n(int n) {
+  return kIdescBase | ((uint32_t)(n >> 3) << 17);
+}
 
 struct LinGeom {
   long long rows;  // R = B * N
@@ -182,6 +184,12 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
   const int n0 = (int)(blockIdx.x % n_tiles) * BN;
   const long long m0 = (long long)(blockIdx.x / n_tiles) * BM;
   const bool two = n0 + BNH < geom.nout;  // the tile's second half holds outputs
+  // MMA widths of the two halves: the valid columns rounded up to 16, so a
+  // narrow last tile does not multiply zero-filled W rows
+  const int w0 = geom.nout - n0 < BNH ? geom.nout - n0 : BNH;
+  const int w1 = two ? (geom.nout - n0 - BNH < BNH ? geom.nout - n0 - BNH : BNH) : 0;
+  const uint32_t idesc0 = idesc_n((w0 + 15) / 16 * 16);
+  const uint32_t idesc1 = idesc_n(two ? (w1 + 15) / 16 * 16 : 16);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -252,7 +260,7 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes = 2 descriptor units per step
             umma_bf16(tmem_d + (uint32_t)(h * BNH), ad + 2u * (uint64_t)k, bd + 2u * (uint64_t)k,
-                      kIdesc, (kt > 0 || k > 0) ? 1u : 0u);
+                      h == 0 ? idesc0 : idesc1, (kt > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(empty_bar(s));
       }

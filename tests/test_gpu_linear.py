@@ -48,6 +48,8 @@ def _reference(w, x, a, b, wt, bias):
     (1000, 3072, 8, 768, True),   # the KAT-B second-linear shape, ragged rows
     (200, 1536, 16, 200, False),  # n_out not a multiple of 64: the store box is clipped
     (130, 160, 20, 520, True),    # d_g 8 (many groups per K step), n_out just past a tile
+    (300, 1536, 8, 384, True),    # second half 128 wide (narrower MMA)
+    (200, 512, 8, 296, False),    # second half 40 wide: MMA width 48, store clipped at 296
 ])
 def test_fused_linear_matches_oracle(rows, d, n_g, nout, with_bias):
     w, x, a, b, wt, bias = _case(rows, d, n_g, nout)
