@@ -272,3 +272,26 @@ def test_fused_recompute_rejects_overlapping_y():
         st = grk.grkan_forward_backward(tx, tdy, ta, tb, y, dx, dA, dB, w.rows, 1, w.d, w.n_g,
                                         w.m, w.n, w.dtype, ws, wsb)
         assert st == 7  # GRKAN_ERR_ALIAS
+
+
+def test_concurrent_calls_on_two_streams():
+    """Two backward calls with their own workspaces, enqueued on two streams so
+    that the kernels may run at the same time, give the bits of the same calls
+    made one after the other (the kernels share no state besides the error
+    word)."""
+    cases = [case_data("kat_b_ragged"), case_data("stress_ng64")]
+    devs = [_dev(c[0], *c[1:5]) for c in cases]
+    ref = [grk.backward(tx, tdy, ta, tb, c[0].n_g) for c, (tx, tdy, ta, tb) in zip(cases, devs)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for _ in range(3):
+        outs = []
+        for s, c, (tx, tdy, ta, tb) in zip(streams, cases, devs):
+            with torch.cuda.stream(s):
+                outs.append(grk.backward(tx, tdy, ta, tb, c[0].n_g))
+        for s in streams:
+            s.synchronize()
+        for got, want in zip(outs, ref):
+            for u, v in zip(got, want):
+                assert torch.equal(u, v)
+    assert grk.grkan_device_error()[1] == 0
