@@ -605,7 +605,8 @@ struct Cursor3 {
 
 // --- forward -------------------------------------------------------------------------
 // Work items are boxes (row block, group, column box), taken by warp gw of the
-// grid as item gw, gw + total warps, ... in row-block-major order.
+// grid (numbered warp-major) as item gw, gw + total warps, ... in
+// row-block-major order.
 
 
 template <class IO, int M, int N>
@@ -624,7 +625,10 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * S_::kFwdStages;
   const long long row_blocks = (geom.rows + geom.SCw - 1) / geom.SCw;
-  const long long gw = (long long)blockIdx.x * kWarps + warp;
+  // warp-major numbering: consecutive work items go to different SMs, so the
+  // items left over after whole rounds spread over every SM instead of
+  // filling the first SMs' warps
+  const long long gw = (long long)warp * gridDim.x + blockIdx.x;
   const long long GW = (long long)gridDim.x * kWarps;
 
   if (lane == 0) {
@@ -727,10 +731,11 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
 }
 
 // --- backward ------------------------------------------------------------------------
-// Units (tile, g) (tile = S rows) are taken by warp gw of the grid as unit
-// gw, gw + total warps, ... in tile-major order; a unit's boxes are its row
-// blocks (SCw rows) times the group's column boxes. The partial sum of unit
-// (tile, g), coefficient k goes to ws[(g * 10 + k) * ws_T + ws_tile0 + tile].
+// Units (tile, g) (tile = S rows) are taken by warp gw of the grid (numbered
+// warp-major, gw = warp * grid + CTA) as unit gw, gw + total warps, ... in
+// tile-major order; a unit's boxes are its row blocks (SCw rows) times the
+// group's column boxes. The partial sum of unit (tile, g), coefficient k goes to
+// ws[(g * K + k) * ws_T + ws_tile0 + tile], K = m + 1 + n.
 
 
 // Row blocks of tile `tile`: ceil(min(S, rows - tile * S) / SCw); only the last
@@ -765,7 +770,10 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   const bool use_tab = geom.n_g <= kTableGroups;
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * S_::kBwdStages;
-  const long long gw = (long long)blockIdx.x * kWarps + warp;
+  // warp-major numbering: consecutive work items go to different SMs, so the
+  // items left over after whole rounds spread over every SM instead of
+  // filling the first SMs' warps
+  const long long gw = (long long)warp * gridDim.x + blockIdx.x;
   const long long GW = (long long)gridDim.x * kWarps;
 
   if (lane == 0) {
