@@ -2,21 +2,24 @@
 //
 // Work decomposition: (row tile x group) units as in the FlashKAT backward
 // ("FlashKAT ...", paper notes, section "3. FlashKAT kernel restructuring
-// (Algorithm 2)"), realised as a persistent grid of one 16-warp CTA per SM that
-// walks the unit list in a fixed stride. A unit is split into chunks of SC rows
-// x d_g channels (24 KiB of one tensor) that stream through a ring of shared-
-// memory stages filled by 2-D TMA tile loads:
-//   - thread 0 also acts as the issuer: it stages the group's coefficients in
-//     the stage header and issues the loads, keeping the ring full by refilling
-//     the stage of chunk q-1 (once every warp has read it) when it starts q;
-//   - every warp reads its vectors of the chunk into registers, releases the
-//     stage, evaluates the rational function on pairs of elements with packed
-//     float32x2 arithmetic, and writes y or dx with 16-byte global stores;
-//   - the backward keeps the ten coefficient-gradient sums in registers; at the
-//     end of a unit they are folded in a fixed order through shared memory and
-//     warp shuffles into one float32 partial per (unit, coefficient) in the
-//     workspace -- no atomics (section "3. ...": accumulate inside the block,
-//     one global write per block).
+// (Algorithm 2)"), realised as a persistent grid of one 16-warp CTA per SM in
+// which every warp runs its own pipeline:
+//   - a warp owns a ring of shared-memory stages (one 2-D TMA box of every input
+//     tensor each) with its own full / empty mbarriers; its lane 0 issues the
+//     box loads `stages` boxes ahead and refills a slot as soon as the warp has
+//     read it; nothing couples the warps of a CTA after start-up, so one warp's
+//     loads overlap another's arithmetic;
+//   - work items (forward: boxes; backward: units of 8 boxes) are taken by the
+//     warps in a fixed stride over a warp-major numbering, with division-free
+//     mixed-radix cursors;
+//   - the lanes evaluate the rational function on pairs of elements with packed
+//     float32x2 arithmetic from coefficients kept in a CTA-wide table, and write
+//     y or dx with 16-byte streaming stores;
+//   - the backward keeps the m + 1 + n coefficient-gradient sums in registers;
+//     at the end of a unit the warp folds them in a fixed order (recursive
+//     halving over shuffles) into one float32 partial per (unit, coefficient)
+//     in the workspace -- no atomics (section "3. ...": accumulate inside the
+//     block, one global write per block).
 // Every wait is bounded: a wait that runs out records a code in
 // g_grkan_device_error and the kernel winds down instead of hanging.
 #pragma once
