@@ -54,13 +54,21 @@ struct TmaGeom {
 };
 
 // Launch shape (compile-time; the defaults are the tuned configuration).
-// One CTA of kWarps independent warps per SM. Every warp owns, per element
+// One CTA of independent warps per SM (16 for the forward; for the backward 16 in
+// float32, HBM-bound, and 12 in bf16, whose arithmetic-bound loop runs faster with
+// up to 168 registers per thread). Every warp owns, per element
 // type, a ring of forward stages (one box of x each) and of backward stages
 // (one box of x and one of dy each). float32 rows are HBM-bound: smaller boxes,
 // deeper rings. The bf16 backward is bound by arithmetic issue: 3 KiB boxes read
 // in three passes of two 16-byte vectors per lane, two stages.
-#ifndef GRK_WARPS
-#define GRK_WARPS 16
+#ifndef GRK_FWD_WARPS
+#define GRK_FWD_WARPS 16
+#endif
+#ifndef GRK_F32_BWD_WARPS
+#define GRK_F32_BWD_WARPS 16
+#endif
+#ifndef GRK_BF16_BWD_WARPS
+#define GRK_BF16_BWD_WARPS 12
 #endif
 #ifndef GRK_F32_FWD_VEC
 #define GRK_F32_FWD_VEC 6
@@ -93,8 +101,8 @@ struct TmaGeom {
 #define GRK_BF16_BWD_STAGES 2
 #endif
 
-constexpr int kWarps = GRK_WARPS;
-constexpr int kThreads = kWarps * 32;
+constexpr int kFwdWarps = GRK_FWD_WARPS;  // forward: 16 warps x 128 registers
+constexpr int kFwdThreads = kFwdWarps * 32;
 
 template <class IO>
 struct Shape;
@@ -105,6 +113,7 @@ struct Shape<IoF32> {
   static constexpr int kBwdVec = GRK_F32_BWD_VEC;        // vectors per lane and tensor in one pass
   static constexpr int kBwdHalves = GRK_F32_BWD_HALVES;  // passes over a backward box
   static constexpr int kBwdStages = GRK_F32_BWD_STAGES;  // backward ring depth
+  static constexpr int kBwdWarps = GRK_F32_BWD_WARPS;    // backward warps per CTA
 };
 template <>
 struct Shape<IoBF16> {
@@ -113,6 +122,7 @@ struct Shape<IoBF16> {
   static constexpr int kBwdVec = GRK_BF16_BWD_VEC;
   static constexpr int kBwdHalves = GRK_BF16_BWD_HALVES;
   static constexpr int kBwdStages = GRK_BF16_BWD_STAGES;
+  static constexpr int kBwdWarps = GRK_BF16_BWD_WARPS;
 };
 template <class IO>
 constexpr unsigned fwd_box_bytes() {
@@ -613,7 +623,7 @@ struct Cursor3 {
 
 
 template <class IO, int M, int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
   using S_ = Shape<IO>;
@@ -623,7 +633,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   const int warp = threadIdx.x >> 5;
   const WarpLayout L(geom.box_bytes, 1, S_::kFwdStages);
   unsigned char* base = smem + warp * L.per_warp;
-  float* ctab = reinterpret_cast<float*>(smem + kWarps * L.per_warp);
+  float* ctab = reinterpret_cast<float*>(smem + kFwdWarps * L.per_warp);
   const bool use_tab = geom.n_g <= kTableGroups;
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * S_::kFwdStages;
@@ -632,7 +642,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
   // items left over after whole rounds spread over every SM instead of
   // filling the first SMs' warps
   const long long gw = (long long)warp * gridDim.x + blockIdx.x;
-  const long long GW = (long long)gridDim.x * kWarps;
+  const long long GW = (long long)gridDim.x * kFwdWarps;
 
   if (lane == 0) {
     for (int s = 0; s < S_::kFwdStages; ++s) {
@@ -752,7 +762,7 @@ __device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile)
 // kFull: every 16-byte vector slot of a lane holds box data (the box is exactly
 // 32 * NV vectors), so the loads need no guard.
 template <class IO, int M, int N, bool kWithY, bool kFull>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Shape<IO>::kBwdWarps * 32, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
         typename IO::T* __restrict__ dx, typename IO::T* __restrict__ yout,
         const float* __restrict__ a,
@@ -769,7 +779,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   const int warp = threadIdx.x >> 5;
   const WarpLayout L(geom.box_bytes, 2, S_::kBwdStages);
   unsigned char* base = smem + warp * L.per_warp;
-  float* ctab = reinterpret_cast<float*>(smem + kWarps * L.per_warp);
+  float* ctab = reinterpret_cast<float*>(smem + S_::kBwdWarps * L.per_warp);
   const bool use_tab = geom.n_g <= kTableGroups;
   const uint32_t full0 = smem_addr(base + L.bar_off);
   const uint32_t empty0 = full0 + 8 * S_::kBwdStages;
@@ -777,7 +787,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   // items left over after whole rounds spread over every SM instead of
   // filling the first SMs' warps
   const long long gw = (long long)warp * gridDim.x + blockIdx.x;
-  const long long GW = (long long)gridDim.x * kWarps;
+  const long long GW = (long long)gridDim.x * S_::kBwdWarps;
 
   if (lane == 0) {
     for (int s = 0; s < S_::kBwdStages; ++s) {
@@ -998,16 +1008,16 @@ inline cudaError_t ensure_smem(unsigned bytes) {
   return e;
 }
 
-// Shared memory of a launch: kWarps per-warp regions of the largest box, then
+// Shared memory of a launch: one region per warp for the largest box, then
 // the coefficient table.
 template <class IO, int M, int N>
 inline unsigned fwd_smem_bytes() {
-  return kWarps * WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages).per_warp +
+  return kFwdWarps * WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages).per_warp +
          coef_table_bytes<M, N>();
 }
 template <class IO, int M, int N>
 inline unsigned bwd_smem_bytes() {
-  return kWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp +
+  return Shape<IO>::kBwdWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp +
          coef_table_bytes<M, N>();
 }
 
@@ -1018,7 +1028,7 @@ inline cudaError_t launch_fwd_tma_t(const TmaGeom& g, const CUtensorMap& mx, voi
   const unsigned smem = fwd_smem_bytes<IO, M, N>();
   cudaError_t e = ensure_smem<fwd_tma<IO, M, N>>(smem);
   if (e != cudaSuccess) return e;
-  fwd_tma<IO, M, N><<<(unsigned)grid, kThreads, smem, st>>>(mx, (typename IO::T*)y, a, b, g);
+  fwd_tma<IO, M, N><<<(unsigned)grid, kFwdThreads, smem, st>>>(mx, (typename IO::T*)y, a, b, g);
   return cudaGetLastError();
 }
 
@@ -1027,7 +1037,7 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   if (g.box_bytes > fwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long items = ((g.rows + g.SCw - 1) / g.SCw) * g.n_g * g.nbox;
   long long grid = sms;
-  if (grid * kWarps > items) grid = (items + kWarps - 1) / kWarps;
+  if (grid * kFwdWarps > items) grid = (items + kFwdWarps - 1) / kFwdWarps;
 #define GRK_FWD_CASE(M, N)                                                          \
   if (g.m == M && g.n == N)                                                         \
     return bf16 ? launch_fwd_tma_t<IoBF16, M, N>(g, mx, y, a, b, grid, st)          \
@@ -1044,7 +1054,7 @@ inline cudaError_t launch_bwd_tma_t(const TmaGeom& g, const CUtensorMap& mx,
   const unsigned smem = bwd_smem_bytes<IO, M, N>();
   cudaError_t e = ensure_smem<bwd_tma<IO, M, N, kWithY, kFull>>(smem);
   if (e != cudaSuccess) return e;
-  bwd_tma<IO, M, N, kWithY, kFull><<<(unsigned)grid, kThreads, smem, st>>>(
+  bwd_tma<IO, M, N, kWithY, kFull><<<(unsigned)grid, Shape<IO>::kBwdWarps * 32, smem, st>>>(
       mx, mdy, (typename IO::T*)dx, (typename IO::T*)y, a, b, ws, g);
   return cudaGetLastError();
 }
@@ -1074,8 +1084,9 @@ inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
                                   const float* b, float* ws, int sms, cudaStream_t st) {
   if (g.box_bytes > bwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long units = g.T * g.n_g;
+  const int warps = bf16 ? Shape<IoBF16>::kBwdWarps : Shape<IoF32>::kBwdWarps;
   long long grid = sms;
-  if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
+  if (grid * warps > units) grid = (units + warps - 1) / warps;
 #define GRK_BWD_CASE(M, N)                                                              \
   if (g.m == M && g.n == N)                                                             \
     return bf16 ? launch_bwd_tma_io<IoBF16, M, N>(g, mx, mdy, dx, y, a, b, ws, grid, st) \
