@@ -20,6 +20,7 @@ __all__ = [
     "grkan_step_host", "grkan_step_host_scratch_bytes", "grkan_forward_backward",
     "grkan_backward_atomic", "ATOMIC_PER_ELEMENT", "ATOMIC_PER_BLOCK",
     "grkan_linear_forward", "linear_forward",
+    "grkan_linear_backward", "grkan_linear_backward_workspace_bytes", "linear_backward",
     "forward_backward",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
     "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
@@ -70,6 +71,10 @@ def _load():
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
         "grkan_linear_forward": (S, [P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I64,
                                      ctypes.c_int, P]),
+        "grkan_linear_backward_workspace_bytes": (SZ, [I64, I64, I64, I32, I32, I32, I64,
+                                                       ctypes.c_int]),
+        "grkan_linear_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I64,
+                                      ctypes.c_int, P, SZ, P]),
         "grkan_backward_atomic": (S, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                       ctypes.c_int, I32, I32, P]),
         "grkan_forward_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
@@ -198,6 +203,40 @@ def linear_forward(x, a, b, n_g, W, bias=None, stream=None):
     _check(grkan_linear_forward(x, a, b, W, bias, out, B, N, d, n_g, m, n, nout, dt, stream),
            "grkan_linear_forward")
     return out
+
+
+def grkan_linear_backward_workspace_bytes(B, N, d, n_g, m, n, nout, dtype):
+    return lib().grkan_linear_backward_workspace_bytes(B, N, d, n_g, m, n, nout, dtype)
+
+
+def grkan_linear_backward(x, dout, W, a, b, dx, dA, dB, B, N, d, n_g, m, n, nout, dtype,
+                          workspace, workspace_bytes, stream=None):
+    return lib().grkan_linear_backward(_ptr(x), _ptr(dout), _ptr(W), _ptr(a), _ptr(b), _ptr(dx),
+                                       _ptr(dA), _ptr(dB), B, N, d, n_g, m, n, nout, dtype,
+                                       _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def linear_backward(x, dout, W, a, b, n_g, dx=None, dA=None, dB=None, workspace=None,
+                    stream=None):
+    """(dx, dA, dB) of GR-KAN followed by a linear layer, from the layer output's
+    gradient dout (B, N, nout) bf16 and the weight W (nout, d) bf16."""
+    import torch
+    B, N, d, dt = _dims(x, n_g)
+    m, n = _coef(a, b, n_g)
+    nout = W.shape[0]
+    if dx is None:
+        dx = torch.empty_like(x)
+    if dA is None:
+        dA = torch.empty((n_g, m + 1), dtype=torch.float32, device=x.device)
+    if dB is None:
+        dB = torch.empty((n_g, n), dtype=torch.float32, device=x.device)
+    wsb = grkan_linear_backward_workspace_bytes(B, N, d, n_g, m, n, nout, dt)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=x.device)
+    _check(grkan_linear_backward(x, dout, W, a, b, dx, dA, dB, B, N, d, n_g, m, n, nout, dt,
+                                 workspace, workspace.numel() * workspace.element_size(), stream),
+           "grkan_linear_backward")
+    return dx, dA, dB
 
 
 def grkan_backward_atomic(x, dy, a, b, dx, dA, dB, B, N, d, n_g, m, n, dtype, mode, block_rows=0,

@@ -15,6 +15,7 @@
 #include "grkan_common.cuh"
 #include "grkan_generic.cuh"
 #include "grkan_linear.cuh"
+#include "grkan_linear_bwd.cuh"
 #include "grkan_merge.cuh"
 #include "grkan_tma.cuh"
 
@@ -678,6 +679,115 @@ grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* 
     e = cudaGetLastError();
   }
   return cuda_status(e, "grkan_linear_forward launch");
+}
+
+namespace {
+
+// Partial slots of the fused data-gradient kernel per (group, coefficient): one
+// per (128-row tile, 64-channel block of the group, 32-row quarter).
+long long dgrad_slots(const Plan& p) {
+  return ((p.rows + grk::lin::dg::BM - 1) / grk::lin::dg::BM) * (p.dg / 64) * 4;
+}
+
+// Shape checks of grkan_linear_backward (the plan is valid).
+grkan_status_t dgrad_shape(const Plan& p, int64_t nout) {
+  if (p.dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
+  if (p.m != 5 || p.n != 4) return GRKAN_ERR_DEGREE;
+  if (nout < 0 || nout % 8 != 0 || nout > 0x7fffffffLL || p.dg % 64 != 0 ||
+      p.rows > 0x7fffffffLL || p.d > 0x7fffffffLL)
+    return GRKAN_ERR_SHAPE;
+  if (p.rows > 0 && p.d > 0 && (long long)p.n_g * dgrad_slots(p) > (1LL << 31) - 1)
+    return GRKAN_ERR_SHAPE;
+  return GRKAN_OK;
+}
+
+}  // namespace
+
+size_t grkan_linear_backward_workspace_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g,
+                                             int32_t m, int32_t n, int64_t nout,
+                                             grkan_dtype_t dtype) {
+  Plan p;
+  if (make_plan(B, N, d, n_g, m, n, dtype, &p) != GRKAN_OK || dgrad_shape(p, nout) != GRKAN_OK)
+    return 0;
+  if (p.rows == 0 || p.d == 0 || nout == 0) return 0;
+  return (size_t)dgrad_slots(p) * (size_t)p.n_g * (size_t)p.K * sizeof(float);
+}
+
+grkan_status_t grkan_linear_backward(const void* x, const void* dout, const void* W,
+                                     const float* a, const float* b, void* dx, float* dA,
+                                     float* dB, int64_t B, int64_t N, int64_t d, int32_t n_g,
+                                     int32_t m, int32_t n, int64_t nout, grkan_dtype_t dtype,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s != GRKAN_OK) return s;
+  if ((s = dgrad_shape(p, nout)) != GRKAN_OK) return s;
+  if (!dA || !dB) return GRKAN_ERR_NULL;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t xbytes = (size_t)p.rows * (size_t)p.d * 2;
+  if (p.rows == 0 || p.d == 0 || nout == 0) {
+    // no rows: empty sums; no output features: dy = 0, so dx = 0 and the sums are 0
+    cudaError_t e = cudaSuccess;
+    if (xbytes > 0) {
+      if (!dx) return GRKAN_ERR_NULL;
+      e = cudaMemsetAsync(dx, 0, xbytes, st);
+    }
+    if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, sizeof(float) * p.n_g * (p.m + 1), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, sizeof(float) * p.n_g * p.n, st);
+    return cuda_status(e, "grkan_linear_backward zeroing");
+  }
+  if (!x || !dout || !W || !dx) return GRKAN_ERR_NULL;
+  if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+  if (!aligned16(x) || !aligned16(dout) || !aligned16(W) || !aligned16(dx))
+    return GRKAN_ERR_SHAPE;
+  const long long T = dgrad_slots(p);
+  const size_t ws_bytes = (size_t)T * (size_t)p.n_g * (size_t)p.K * sizeof(float);
+  if (!workspace || workspace_bytes < ws_bytes || !aligned16(workspace)) return GRKAN_ERR_WORKSPACE;
+  const size_t dobytes = (size_t)p.rows * (size_t)nout * 2;
+  const size_t wbytes = (size_t)nout * (size_t)p.d * 2;
+  if (overlaps(dx, xbytes, x, xbytes) || overlaps(dx, xbytes, dout, dobytes) ||
+      overlaps(dx, xbytes, W, wbytes) || overlaps(workspace, ws_bytes, x, xbytes) ||
+      overlaps(workspace, ws_bytes, dout, dobytes) || overlaps(workspace, ws_bytes, W, wbytes) ||
+      overlaps(workspace, ws_bytes, dx, xbytes))
+    return GRKAN_ERR_ALIAS;
+  namespace dg = grk::lin::dg;
+  CUtensorMap mdo, mw, mx, mdx;
+  if (!make_map_bf16(&mdo, dout, (uint64_t)nout, (uint64_t)p.rows, dg::BK, dg::BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mw, W, (uint64_t)p.d, (uint64_t)nout, 64, dg::BK,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, 32, dg::BM,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_bf16(&mdx, dx, (uint64_t)p.d, (uint64_t)p.rows, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+    return GRKAN_ERR_CUDA;
+  dg::DgGeom g;
+  g.rows = p.rows;
+  g.d = (int)p.d;
+  g.nout = (int)nout;
+  g.dg = (int)p.dg;
+  g.n_g = p.n_g;
+  g.kt = (int)((nout + dg::BK - 1) / dg::BK);
+  g.n_ct = (int)((p.d + dg::BN - 1) / dg::BN);
+  g.n_tiles = ((p.rows + dg::BM - 1) / dg::BM) * g.n_ct;
+  g.ws_T = T;
+  g.nbg = (int)(p.dg / 64);
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = grk::ensure_smem<dg::linear_dgrad>(dg::Layout::kAlloc);
+  if (e == cudaSuccess) {
+    const long long grid = g.n_tiles < sms ? g.n_tiles : sms;
+    dg::linear_dgrad<<<(unsigned)grid, dg::kThreads, dg::Layout::kAlloc, st>>>(
+        mdo, mw, mx, mdx, a, b, (float*)workspace, g);
+    e = cudaGetLastError();
+  }
+  if ((s = cuda_status(e, "grkan_linear_backward launch")) != GRKAN_OK) return s;
+  Plan pm = p;
+  pm.T = T;
+  return cuda_status(launch_merge(pm, (const float*)workspace, dA, dB, nullptr, st),
+                     "grkan_linear_backward merge");
 }
 
 grkan_status_t grkan_merge_ranks(const double* gathered, int32_t world, float* dA, float* dB,

@@ -148,6 +148,37 @@ GRKAN_API grkan_status_t grkan_linear_forward(const void* x, const float* a, con
                                               int32_t m, int32_t n, int64_t nout,
                                               grkan_dtype_t dtype, void* stream);
 
+/* The GR-KAN backward fused into the data-gradient product of the linear layer
+ * that follows the activation (the backward of grkan_linear_forward without its
+ * weight gradient):
+ *   dy[r, c] = sum_o dout[r, o] W[o, c]      (float32, on the tensor cores)
+ *   dx, dA, dB = grkan_backward(x, dy)        (with this float32 dy)
+ * dy is the product's accumulator and never goes to memory. x: bf16 (B*N rows x
+ * d), row-major. dout: bf16 (B*N x nout), row-major (the layer output's
+ * gradient). W: bf16 (nout x d), row-major (the linear layer's weight). dx: bf16
+ * like x, overwritten; dA (n_g x 6), dB (n_g x 4) float32, overwritten. dA and dB
+ * are reduced in a fixed order, as grkan_backward's (the same bits on every
+ * run). workspace: device memory of at least
+ * grkan_linear_backward_workspace_bytes (which returns 0 for shapes this call
+ * rejects and when nothing needs reducing), 16-byte aligned, owned by the caller
+ * and free for the call's duration on its stream. nout == 0 gives dx = 0 and
+ * zero gradients; B*N == 0 gives zero gradients.
+ * Requires dtype GRKAN_BF16 (else GRKAN_ERR_DTYPE), (m, n) = (5, 4) (else
+ * GRKAN_ERR_DEGREE), d_g % 64 == 0, nout % 8 == 0 and 16-byte aligned x, dout,
+ * W, dx (else GRKAN_ERR_SHAPE); dx and the workspace may not overlap x, dout, W
+ * or each other (GRKAN_ERR_ALIAS). */
+GRKAN_API size_t grkan_linear_backward_workspace_bytes(int64_t B, int64_t N, int64_t d,
+                                                       int32_t n_g, int32_t m, int32_t n,
+                                                       int64_t nout, grkan_dtype_t dtype);
+
+GRKAN_API grkan_status_t grkan_linear_backward(const void* x, const void* dout, const void* W,
+                                               const float* a, const float* b, void* dx,
+                                               float* dA, float* dB, int64_t B, int64_t N,
+                                               int64_t d, int32_t n_g, int32_t m, int32_t n,
+                                               int64_t nout, grkan_dtype_t dtype,
+                                               void* workspace, size_t workspace_bytes,
+                                               void* stream);
+
 /* Coefficient gradients accumulated with float32 atomic adds, the two schemes
  * that "FlashKAT: Understanding and Addressing Performance Bottlenecks in the
  * Kolmogorov-Arnold Transformer" compares (paper notes, sections "2. The
