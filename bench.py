@@ -367,7 +367,35 @@ def main():
                   "fused_TFLOP/s": fl / (f_ms * 1e-3) / 1e12,
                   "note": "grkan_linear_forward vs grkan_forward + torch.matmul (cuBLAS), "
                           "no bias; not part of the timed step"}
-        del Wl, outl
+
+        # its backward: dy = dout W on the tensor cores with the GR-KAN backward as
+        # the epilogue, against torch.matmul (cuBLAS, bf16 dy) + grkan_backward;
+        # alternated three times, medians
+        dout = (torch.randn(B * N, nout, device=dev, generator=gen) * 1e-2).to(torch.bfloat16)
+        dyl = torch.empty_like(dy)
+        wslb = grk.grkan_linear_backward_workspace_bytes(B, N, d, n_g, m, n, nout, dt)
+        wsl = torch.empty(max(wslb, 16), dtype=torch.uint8, device=dev)
+
+        def lbw_fused():
+            check(grk.grkan_linear_backward(x, dout, Wl, a, b, dx, dA, dB, B, N, d, n_g, m, n,
+                                            nout, dt, wsl, wslb, sp), "linear_backward")
+
+        def lbw_unfused():
+            torch.matmul(dout, Wl, out=dyl.view(B * N, d))
+            check(grk.grkan_backward(x, dyl, a, b, dx, dA, dB, B, N, d, n_g, m, n, dt, ws, wsb,
+                                     sp), "backward")
+
+        fb, ub = [], []
+        for _ in range(3):
+            fb.append(timed(lbw_fused))
+            ub.append(timed(lbw_unfused))
+        fb_ms, ub_ms = sorted(fb)[1], sorted(ub)[1]
+        linear["backward"] = {
+            "fused_ms": fb_ms, "unfused_ms": ub_ms,
+            "fused_TFLOP/s": fl / (fb_ms * 1e-3) / 1e12,
+            "note": "grkan_linear_backward (dout W + GR-KAN backward epilogue, CTA pairs) vs "
+                    "torch.matmul (cuBLAS) + grkan_backward; weight gradient not included"}
+        del Wl, outl, dout, dyl, wsl
 
     # end to end through the C ABI's host-buffer entry point: pinned inputs in,
     # y, dx and dA/dB out, copies inside the timed region (chunks streamed over

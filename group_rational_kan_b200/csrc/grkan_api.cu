@@ -689,6 +689,43 @@ long long dgrad_slots(const Plan& p) {
   return ((p.rows + grk::lin::dg::BM - 1) / grk::lin::dg::BM) * (p.dg / 64) * 4;
 }
 
+// CTA pairs of the fused data-gradient kernel that are resident at once on the
+// current device (a pair needs two SMs of one GPC), looked up once per device.
+cudaError_t dgrad_pairs(int* out) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+    *out = cached[dev];
+    return cudaSuccess;
+  }
+  namespace dg = grk::lin::dg;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(sms / 2 * 2), 1, 1);
+  cfg.blockDim = dim3(dg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = dg::Layout::kAlloc;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, dg::linear_dgrad, &cfg);
+  if (e != cudaSuccess) return e;
+  if (n < 1) n = 1;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  *out = n;
+  return cudaSuccess;
+}
+
 // Shape checks of grkan_linear_backward (the plan is valid).
 grkan_status_t dgrad_shape(const Plan& p, int64_t nout) {
   if (p.dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
@@ -755,8 +792,8 @@ grkan_status_t grkan_linear_backward(const void* x, const void* dout, const void
   CUtensorMap mdo, mw, mx, mdx;
   if (!make_map_bf16(&mdo, dout, (uint64_t)nout, (uint64_t)p.rows, dg::BK, dg::BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_bf16(&mw, W, (uint64_t)p.d, (uint64_t)nout, 64, dg::BK,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mw, W, (uint64_t)p.d, (uint64_t)nout, 32, dg::BK,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map_bf16(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, 32, dg::BM,
                      CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map_bf16(&mdx, dx, (uint64_t)p.d, (uint64_t)p.rows, 32, 32,
@@ -770,18 +807,28 @@ grkan_status_t grkan_linear_backward(const void* x, const void* dout, const void
   g.n_g = p.n_g;
   g.kt = (int)((nout + dg::BK - 1) / dg::BK);
   g.n_ct = (int)((p.d + dg::BN - 1) / dg::BN);
-  g.n_tiles = ((p.rows + dg::BM - 1) / dg::BM) * g.n_ct;
+  g.n_tiles = ((p.rows + 2 * dg::BM - 1) / (2 * dg::BM)) * g.n_ct;
+  g.n_mt = (p.rows + dg::BM - 1) / dg::BM;
   g.ws_T = T;
   g.nbg = (int)(p.dg / 64);
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess) e = grk::ensure_smem<dg::linear_dgrad>(dg::Layout::kAlloc);
+  cudaError_t e = grk::ensure_smem<dg::linear_dgrad>(dg::Layout::kAlloc);
+  int pairs = 0;
+  if (e == cudaSuccess) e = dgrad_pairs(&pairs);
   if (e == cudaSuccess) {
-    const long long grid = g.n_tiles < sms ? g.n_tiles : sms;
-    dg::linear_dgrad<<<(unsigned)grid, dg::kThreads, dg::Layout::kAlloc, st>>>(
-        mdo, mw, mx, mdx, a, b, (float*)workspace, g);
-    e = cudaGetLastError();
+    if ((long long)pairs > g.n_tiles) pairs = (int)g.n_tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(dg::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = dg::Layout::kAlloc;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dg::linear_dgrad, mdo, mw, mx, mdx, a, b, (float*)workspace, g);
   }
   if ((s = cuda_status(e, "grkan_linear_backward launch")) != GRKAN_OK) return s;
   Plan pm = p;
