@@ -760,16 +760,14 @@ grkan_status_t grkan_linear_backward(const void* x, const void* dout, const void
   if (s != GRKAN_OK) return s;
   if ((s = dgrad_shape(p, nout)) != GRKAN_OK) return s;
   if (!dA || !dB) return GRKAN_ERR_NULL;
-  if (!is_sm100()) return GRKAN_ERR_DEVICE;
   cudaStream_t st = (cudaStream_t)stream;
   const size_t xbytes = (size_t)p.rows * (size_t)p.d * 2;
   if (p.rows == 0 || p.d == 0 || nout == 0) {
     // no rows: empty sums; no output features: dy = 0, so dx = 0 and the sums are 0
+    if (xbytes > 0 && !dx) return GRKAN_ERR_NULL;
+    if (!is_sm100()) return GRKAN_ERR_DEVICE;
     cudaError_t e = cudaSuccess;
-    if (xbytes > 0) {
-      if (!dx) return GRKAN_ERR_NULL;
-      e = cudaMemsetAsync(dx, 0, xbytes, st);
-    }
+    if (xbytes > 0) e = cudaMemsetAsync(dx, 0, xbytes, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, sizeof(float) * p.n_g * (p.m + 1), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, sizeof(float) * p.n_g * p.n, st);
     return cuda_status(e, "grkan_linear_backward zeroing");
@@ -788,6 +786,7 @@ grkan_status_t grkan_linear_backward(const void* x, const void* dout, const void
       overlaps(workspace, ws_bytes, dout, dobytes) || overlaps(workspace, ws_bytes, W, wbytes) ||
       overlaps(workspace, ws_bytes, dx, xbytes))
     return GRKAN_ERR_ALIAS;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
   namespace dg = grk::lin::dg;
   CUtensorMap mdo, mw, mx, mdx;
   if (!make_map_bf16(&mdo, dout, (uint64_t)nout, (uint64_t)p.rows, dg::BK, dg::BM,

@@ -131,3 +131,66 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         grk.lib()
     importlib.reload(grk)
+
+
+def test_linear_backward_argument_errors_need_no_gpu():
+    A = 1 << 20        # x
+    DO = 1 << 28       # dout
+    WT = 1 << 29       # W
+    DX = 1 << 30       # dx
+    WS = 1 << 31       # workspace
+    K = (1 << 32)      # dA, dB, coefficients
+    rows, d, n_g, nout = 300, 768, 4, 576
+    need = grk.grkan_linear_backward_workspace_bytes(1, rows, d, n_g, 5, 4, nout, grk.BF16)
+    # one float32 partial per (128-row tile, 64-channel block of a group, row quarter)
+    assert need == 3 * (192 // 64) * 4 * n_g * 10 * 4
+    assert grk.grkan_linear_backward_workspace_bytes(1, rows, d, n_g, 5, 4, nout, grk.F32) == 0
+    assert grk.grkan_linear_backward_workspace_bytes(1, rows, d, 8, 5, 4, nout, grk.BF16) == 0
+    assert grk.grkan_linear_backward_workspace_bytes(1, rows, d, n_g, 5, 4, 0, grk.BF16) == 0
+
+    def call(x=A, dout=DO, W=WT, a=K, b=K + 64, dx=DX, dA=K + 256, dB=K + 512, rows=rows, d=d,
+             n_g=n_g, m=5, n=4, nout=nout, dtype=grk.BF16, ws=WS, wsb=need):
+        return grk.grkan_linear_backward(x, dout, W, a, b, dx, dA, dB, 1, rows, d, n_g, m, n,
+                                         nout, dtype, ws, wsb, 0)
+
+    assert call(dtype=grk.F32) == DTYPE
+    assert call(m=4) == DEGREE
+    assert call(n_g=8) == SHAPE            # d_g = 96: not a multiple of 64
+    assert call(nout=100) == SHAPE         # nout % 8
+    assert call(nout=-8) == SHAPE
+    assert call(dA=None) == NULL
+    assert call(x=None) == NULL
+    assert call(dout=None) == NULL
+    assert call(W=None) == NULL
+    assert call(a=None) == NULL
+    assert call(x=A + 8) == SHAPE          # 16-byte alignment
+    assert call(ws=None) == WORKSPACE
+    assert call(wsb=need - 4) == WORKSPACE
+    assert call(ws=WS + 4) == WORKSPACE
+    assert call(dx=A + 4096) == ALIAS      # dx overlaps x
+    assert call(dx=DO) == ALIAS            # dx overlaps dout
+    assert call(ws=DX + 4096) == ALIAS     # workspace inside dx
+    assert call(nout=0, dx=None) == NULL   # dx = 0 is written
+    if not _has_gpu():
+        assert call() == DEVICE
+        assert call(nout=0) == DEVICE      # zeroing needs the device too
+
+
+def test_linear_forward_argument_errors_need_no_gpu():
+    A, WT, O = 1 << 20, 1 << 29, 1 << 30
+    K = 1 << 32
+
+    def call(x=A, a=K, b=K + 64, W=WT, bias=None, out=O, d=768, n_g=8, m=5, n=4, nout=576,
+             dtype=grk.BF16):
+        return grk.grkan_linear_forward(x, a, b, W, bias, out, 1, 300, d, n_g, m, n, nout, dtype,
+                                        0)
+
+    assert call(dtype=grk.F32) == DTYPE
+    assert call(n=3) == DEGREE
+    assert call(d=760, n_g=8) == SHAPE     # d % 32
+    assert call(nout=100) == SHAPE         # nout % 8
+    assert call(x=None) == NULL
+    assert call(W=WT + 8) == SHAPE         # alignment
+    assert call(out=A + 64) == ALIAS       # out overlaps x
+    if not _has_gpu():
+        assert call() == DEVICE
