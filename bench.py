@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--m", type=int, default=None, help="numerator degree (degree sweeps)")
     ap.add_argument("--n", type=int, default=None, help="denominator degree (degree sweeps)")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -172,8 +174,8 @@ def run_reference(args, w):
         return
     import oracle
     orc = oracle.Oracle()
-    # size one step so that warmup + steps take about two minutes in all
-    budget = 120.0 / max(args.steps + args.warmup, 1)
+    # size one step so that warmup + steps take about --ref-budget seconds in all
+    budget = args.ref_budget / max(args.steps + args.warmup, 1)
     rows, dt, cores = oracle_rate(w, min(budget, 2.0))
     per_row = dt / rows
     rows = max(1, min(w.rows, int(budget / per_row)))
