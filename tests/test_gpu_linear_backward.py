@@ -110,6 +110,9 @@ def _check(x, dout, W, a, b, n_g, got_dx, dA, dB):
     (200, 320, 5, 128),     # d_g 64: last column tile 128 wide (N 128, one warp column idle)
     (260, 448, 7, 200),     # last column tile 64 wide, last K step partly past nout
     (130, 1536, 8, 8),      # nout 8: one K step, mostly zero-filled
+    (300, 6144, 96, 64),    # 96 groups: coefficients from global memory, not the table
+    (1, 384, 2, 64),        # one row: the pair's second CTA and 127 rows are past the end
+    (256, 384, 2, 4096),    # 64 K steps through the ring
 ])
 def test_fused_linear_backward_matches_oracle(rows, d, n_g, nout):
     w, x, a, b, dout, W = _case(rows, d, n_g, nout)
