@@ -4,10 +4,12 @@ against FlashKAT's per-block accumulation), measured against the fp64 oracle on
 the same inputs, next to this library's two-stage fixed-order reduction.
 
 Pinned here: dx of both atomic schemes is the generic backward's, bit for bit;
-the per-element scheme's mean absolute error is at least ten times that of the
-per-block scheme and of the two-stage reduction (the direction of the paper's
-table); the two-stage result stays within the library's tolerance and is
-identical from run to run."""
+the per-element scheme's mean absolute error is well above the per-block
+scheme's (at least four times: the ratio depends on the order in which the
+atomics land and was measured between 9.9 and about 15) and at least ten times
+the two-stage reduction's, and the per-block scheme's is above the two-stage
+reduction's (the direction of the paper's table); the two-stage result stays
+within the library's tolerance and is identical from run to run."""
 import numpy as np
 import pytest
 import torch
@@ -70,8 +72,9 @@ def test_atomic_schemes_against_the_two_stage_reduction(name, rows):
           (w.name, w.rows))
     for label, (mae, var, rel, same) in table.items():
         print("  %-12s %.3e %.3e %.3e %s" % (label, mae, var, rel, same))
-    assert table["per_element"][0] > 10 * table["per_block"][0]
+    assert table["per_element"][0] > 4 * table["per_block"][0]
     assert table["per_element"][0] > 10 * table["two_stage"][0]
+    assert table["per_block"][0] > table["two_stage"][0]
     assert table["two_stage"][3]
     _, dA, dB = runs["two_stage"][0]
     check_coef(dA.cpu().numpy(), dB.cpu().numpy(), ref, what=w.name)
