@@ -23,12 +23,14 @@ __all__ = [
     "grkan_linear_backward", "grkan_linear_backward_workspace_bytes", "linear_backward",
     "forward_backward",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
-    "grkan_status_string", "grkan_abi_version", "grkan_last_error", "forward", "backward", "workspace_bytes",
+    "grkan_status_string", "grkan_abi_version", "grkan_last_error", "grkan_selftest_wait_timeout",
+    "DEVICE_ERROR_SELFTEST", "forward", "backward", "workspace_bytes",
 ]
 
 F32, BF16 = 0, 1
 FLAG_GENERIC = 1
 NOALLOC_WORKSPACE_BYTES = 4 << 20  # GRKAN_NOALLOC_WORKSPACE_BYTES
+DEVICE_ERROR_SELFTEST = 16  # GRKAN_DEVICE_ERROR_SELFTEST
 ABI_VERSION = 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +90,7 @@ def _load():
         "grkan_backward_path": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, ctypes.c_int, U32]),
         "grkan_device_error": (S, [P, P]),
         "grkan_clear_device_error": (S, [P]),
+        "grkan_selftest_wait_timeout": (S, [U32, P]),
         "grkan_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "grkan_abi_version": (I32, []),
         "grkan_last_error": (ctypes.c_char_p, []),
@@ -279,6 +282,10 @@ def grkan_device_error(stream=None):
     code = ctypes.c_uint32(0)
     st = lib().grkan_device_error(ctypes.addressof(code), _stream(stream))
     return st, int(code.value)
+
+
+def grkan_selftest_wait_timeout(limit_us, stream=None):
+    return lib().grkan_selftest_wait_timeout(limit_us, _stream(stream))
 
 
 def grkan_clear_device_error(stream=None):

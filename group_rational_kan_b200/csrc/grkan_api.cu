@@ -1038,6 +1038,14 @@ grkan_status_t grkan_device_error(uint32_t* code, void* stream) {
   return cuda_status(grk::read_device_error(code, st), "grkan_device_error");
 }
 
+grkan_status_t grkan_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 2000000u) return GRKAN_ERR_SHAPE;
+  if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  static_assert(grk::kErrSelfTest == GRKAN_DEVICE_ERROR_SELFTEST, "error bit");
+  grk::selftest_wait_timeout<<<1, 32, 0, (cudaStream_t)stream>>>(1000ull * limit_us);
+  return cuda_status(cudaGetLastError(), "grkan_selftest_wait_timeout launch");
+}
+
 grkan_status_t grkan_clear_device_error(void* stream) {
   return cuda_status(grk::clear_device_error((cudaStream_t)stream), "grkan_clear_device_error");
 }

@@ -68,8 +68,8 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait_sleep(bar, parity)) {
-    if (global_ns() - t0 > kWaitTimeoutNs) return false;
+  for (unsigned polls = 0; !mbar_try_wait_sleep(bar, parity); ++polls) {
+    if (global_ns() - t0 > kWaitTimeoutNs || polls > kMaxPolls) return false;
   }
   return true;
 }

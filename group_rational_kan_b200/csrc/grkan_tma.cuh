@@ -143,12 +143,15 @@ inline unsigned bwd_box_target(bool bf16) {
 #endif
 constexpr int kBoxesPerUnit = GRK_BOXES_PER_UNIT;  // backward boxes per (tile, group) unit
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+// Backstop: a wait also gives up after this many polls, whatever the timer says.
+constexpr unsigned kMaxPolls = 1u << 26;
 
 // Error codes written to g_grkan_device_error (bit-or).
 constexpr unsigned kErrFullWait = 1u;
 constexpr unsigned kErrEmptyWait = 2u;
 constexpr unsigned kErrReduceWait = 4u;
 constexpr unsigned kErrDrainWait = 8u;
+constexpr unsigned kErrSelfTest = 16u;  // grkan_selftest_wait_timeout's wait ran out
 
 __device__ unsigned int g_grkan_device_error = 0;
 
@@ -204,14 +207,19 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// Wait for the phase with the given parity; false after kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase with the given parity; false after limit_ns (or
+// kMaxPolls polls).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitTimeoutNs) return false;
+  for (unsigned polls = 0; !mbar_try_wait(bar, parity); ++polls) {
+    if (global_ns() - t0 > limit_ns || polls > kMaxPolls) return false;
   }
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitTimeoutNs);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
@@ -1094,6 +1102,21 @@ inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
   GRK_TMA_DEGREES(GRK_BWD_CASE)
 #undef GRK_BWD_CASE
   return cudaErrorNotSupported;
+}
+
+// One warp waits on an mbarrier phase that nothing completes, with the same
+// bounded wait as the pipelined kernels and a short limit: the wait runs out,
+// the kernel records kErrSelfTest and returns, and the context stays usable.
+__global__ void selftest_wait_timeout(unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const bool got = mbar_wait_for(b, 0, limit_ns);  // phase 0 never completes
+  if (!__any_sync(0xffffffffu, got) && threadIdx.x == 0) report(kErrSelfTest);
 }
 
 inline cudaError_t read_device_error(uint32_t* out, cudaStream_t st) {

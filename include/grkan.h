@@ -295,6 +295,14 @@ GRKAN_API int32_t grkan_backward_path(const void* x, const void* dy, const void*
 GRKAN_API grkan_status_t grkan_device_error(uint32_t* code, void* stream);
 GRKAN_API grkan_status_t grkan_clear_device_error(void* stream);
 
+/* Self-test of the bounded waits: launches one warp that waits, with the same
+ * wait routine as the pipelined kernels and a limit of limit_us microseconds
+ * (1 .. 2,000,000; else GRKAN_ERR_SHAPE), on an mbarrier phase that nothing
+ * completes. The wait runs out, the kernel ORs GRKAN_DEVICE_ERROR_SELFTEST into
+ * the device error word and returns; the context stays usable. */
+#define GRKAN_DEVICE_ERROR_SELFTEST 16u
+GRKAN_API grkan_status_t grkan_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Human-readable name of a status code (static string). */
 GRKAN_API const char* grkan_status_string(grkan_status_t status);
 

@@ -194,3 +194,10 @@ def test_linear_forward_argument_errors_need_no_gpu():
     assert call(out=A + 64) == ALIAS       # out overlaps x
     if not _has_gpu():
         assert call() == DEVICE
+
+
+def test_selftest_arguments_need_no_gpu():
+    assert grk.grkan_selftest_wait_timeout(0, 0) == SHAPE
+    assert grk.grkan_selftest_wait_timeout(2000001, 0) == SHAPE
+    if not _has_gpu():
+        assert grk.grkan_selftest_wait_timeout(1000, 0) == DEVICE
