@@ -13,6 +13,7 @@ import argparse
 import json
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -100,7 +101,7 @@ class ClockSampler:
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+        self.path = os.path.join(tempfile.gettempdir(), "grkan_clocks_%d.csv" % os.getpid())
 
     def start(self):
         try:
