@@ -69,6 +69,32 @@ struct Layout {
   static constexpr unsigned kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
+// As mbar_try_wait, but the thread may sleep in the instruction until the phase
+// completes (at most kSuspendHintNs per call): a waiting thread issues almost
+// nothing, which leaves the issue slots to the warps that compute.
+constexpr uint32_t kSuspendHintNs = 10000000u;  // 10 ms
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Sleeping wait for the phase with the given parity; false after kWaitTimeoutNs.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (unsigned polls = 0; !mbar_try_wait_sleep(bar, parity); ++polls) {
+    if (global_ns() - t0 > kWaitTimeoutNs || polls > kMaxPolls) return false;
+  }
+  return true;
+}
+
 // --- tcgen05 wrappers ---------------------------------------------------------
 
 __device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
