@@ -16,12 +16,13 @@
 // pair tiles are taken in the order tile = pair + i pairs (row-tile major, so
 // the pairs working at the same time share their dout rows and W columns in L2).
 // In each CTA:
-//   warp 0       lane 0 issues the TMA loads: per tile the CTA's x tile (six
-//                32-channel boxes, 64-byte swizzled, double-buffered), then per
-//                K step of 64 output features its 128 dout rows (K-major,
-//                128-byte swizzled) and its half of the W tile (96 channels as
-//                three 32-channel boxes, channel-major, 64-byte swizzled) into a
-//                ring of stages;
+//   warp 0       lane 0 issues the TMA loads: per K step of 64 output
+//                features the CTA's 128 dout rows (K-major, 128-byte swizzled)
+//                and its half of the W tile (96 channels as three 32-channel
+//                boxes, channel-major, 64-byte swizzled) into a ring of stages,
+//                and per tile, after the first ring's worth of those, the CTA's
+//                x tile (six 32-channel boxes, 64-byte swizzled,
+//                double-buffered);
 //   warp 1       allocates 512 TMEM columns (two 192-column accumulators). In
 //                the leader (rank 0) lane 0 issues four tcgen05.mma (M 256, N
 //                192, K 16; A rows from both CTAs, W from both halves, read
