@@ -7,7 +7,8 @@ source and checks that every planted mistake trips at least one pin.
 
 What pins what:
   y      identity closed form, b = 0 polynomial (exact rationals), exact dyadic
-         brute force, x = 0, bf16 widening, fp64 autograd witness
+         brute force, x = 0, bf16 widening, fp64 autograd witness, numpy's
+         polyval for P and Q with the bound |y| <= |P| (D >= 1)
   dx     identity closed form, x = 0 (dx = dy a_1 under sign(0) = 0), central
          differences of the forward (Richardson), exact dual-number brute force,
          autograd witness
@@ -365,6 +366,31 @@ def pin_noise_scales(orc):
     assert np.all(g["c2_b"] >= g["sabs_b"] ** 2 / nt * (1 - 1e-12))
 
 
+def pin_library_polyval(orc):
+    """y against numpy's own polynomial evaluator for P and Q (b != 0, several
+    degrees, values of x up to 4), and the bound that D = 1 + |Q| >= 1 gives:
+    |y| <= |P(x)|, with equality exactly where Q = 0."""
+    from numpy.polynomial import polynomial as npp
+    rng = np.random.default_rng(21)
+    for (m, n) in ((5, 4), (3, 3), (2, 6), (8, 1)):
+        rows, d, n_g = 7, 12, 3
+        x, dy, a, b = _rand_case(rng, rows, d, n_g, m, n, xs=1.5)
+        x[0, :3] = 0.0
+        y = orc.forward(x, a, b, n_g)
+        dg = d // n_g
+        for g in range(n_g):
+            xs = x[:, g * dg:(g + 1) * dg].astype(np.float64)
+            P = npp.polyval(xs, a[g].astype(np.float64))
+            Q = npp.polyval(xs, np.concatenate([[0.0], b[g].astype(np.float64)]))
+            want = P / (1.0 + np.abs(Q))
+            _close(y[:, g * dg:(g + 1) * dg], want, 1e-13, 1e-300, "y vs polyval (%d,%d)" % (m, n))
+            yg = np.abs(y[:, g * dg:(g + 1) * dg])
+            assert np.all(yg <= np.abs(P) * (1 + 1e-15) + 1e-300), "|y| <= |P|"
+            eq = Q == 0.0
+            assert np.all(yg[eq] == np.abs(P[eq])), "|y| = |P| where Q = 0"
+
+
 ALL_PINS = [pin_identity, pin_polynomial_b0, pin_dyadic_exact, pin_x_zero, pin_bf16_widening,
             pin_fd_dx, pin_fd_dA, pin_fd_dB, pin_autograd, pin_linearity, pin_group_relabel,
-            pin_thread_invariance, pin_sampled_and_extras, pin_ambiguity, pin_noise_scales]
+            pin_thread_invariance, pin_sampled_and_extras, pin_ambiguity, pin_noise_scales,
+            pin_library_polyval]
