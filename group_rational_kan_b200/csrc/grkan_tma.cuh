@@ -59,8 +59,10 @@ struct TmaGeom {
 // up to 168 registers per thread). Every warp owns, per element
 // type, a ring of forward stages (one box of x each) and of backward stages
 // (one box of x and one of dy each). float32 rows are HBM-bound: smaller boxes,
-// deeper rings. The bf16 backward is bound by arithmetic issue: 3 KiB boxes read
-// in three passes of two 16-byte vectors per lane, two stages.
+// deeper rings. The bf16 forward streams 1.5 KiB boxes through four stages
+// (measured faster than 2 KiB x 6). The bf16 backward is bound by arithmetic
+// issue: 3 KiB boxes read in three passes of two 16-byte vectors per lane, two
+// stages.
 #ifndef GRK_FWD_WARPS
 #define GRK_FWD_WARPS 16
 #endif
@@ -86,10 +88,10 @@ struct TmaGeom {
 #define GRK_F32_BWD_STAGES 4
 #endif
 #ifndef GRK_BF16_FWD_VEC
-#define GRK_BF16_FWD_VEC 4
+#define GRK_BF16_FWD_VEC 3
 #endif
 #ifndef GRK_BF16_FWD_STAGES
-#define GRK_BF16_FWD_STAGES 6
+#define GRK_BF16_FWD_STAGES 4
 #endif
 #ifndef GRK_BF16_BWD_VEC
 #define GRK_BF16_BWD_VEC 2
