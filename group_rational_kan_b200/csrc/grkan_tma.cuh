@@ -2,8 +2,8 @@
 //
 // Work decomposition: (row tile x group) units as in the FlashKAT backward
 // ("FlashKAT ...", paper notes, section "3. FlashKAT kernel restructuring
-// (Algorithm 2)"), realised as a persistent grid of one 16-warp CTA per SM in
-// which every warp runs its own pipeline:
+// (Algorithm 2)"), realised as a persistent grid of one CTA per SM (16 warps;
+// 12 for the bf16 backward) in which every warp runs its own pipeline:
 //   - a warp owns a ring of shared-memory stages (one 2-D TMA box of every input
 //     tensor each) with its own full / empty mbarriers; its lane 0 issues the
 //     box loads `stages` boxes ahead and refills a slot as soon as the warp has
