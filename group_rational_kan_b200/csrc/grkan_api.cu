@@ -185,6 +185,10 @@ bool tma_shape_ok(const Plan& p) {
   if (p.rows <= 0 || p.d <= 0) return false;
   if ((p.d * p.es) % 16 != 0 || (p.dg * p.es) % 16 != 0) return false;
   if (p.rows > 0x7fffffffLL || p.d > 0x7fffffffLL) return false;
+  // the kernels keep a lane's byte offsets inside a box (up to scw rows of d
+  // elements) in 32-bit integers
+  const long long scw = p.fbox.scw > p.bbox.scw ? p.fbox.scw : p.bbox.scw;
+  if (scw * p.d * p.es >= 0x7fffffffLL) return false;
   // both boxes exist and every box starts on a 128-byte shared-memory boundary
   // (slots are rounded up to 128 bytes)
   return p.fbox.bw > 0 && p.bbox.bw > 0;
@@ -360,7 +364,8 @@ grkan_status_t do_partials(const Plan& p, const void* x, const void* dy, const f
   if (s != GRKAN_OK) return s;
   if (!ws || ws_bytes < p.ws_bytes || !aligned16(ws)) return GRKAN_ERR_WORKSPACE;
   const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
-  if (bad_alias(x, dx, bytes) || bad_alias(dy, dx, bytes)) return GRKAN_ERR_ALIAS;
+  // dx may replace dy (read before written) but never x, which stays readable
+  if (overlaps(x, bytes, dx, bytes) || bad_alias(dy, dx, bytes)) return GRKAN_ERR_ALIAS;
   if (overlaps(ws, p.ws_bytes, x, bytes) || overlaps(ws, p.ws_bytes, dy, bytes) ||
       overlaps(ws, p.ws_bytes, dx, bytes))
     return GRKAN_ERR_ALIAS;
@@ -563,16 +568,23 @@ grkan_status_t grkan_backward_atomic(const void* x, const void* dy, const float*
   grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
   if (s != GRKAN_OK) return s;
   if (!dA || (p.n > 0 && !dB)) return GRKAN_ERR_NULL;
+  const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
+  if (p.T > 0) {
+    // every check before anything is enqueued
+    if (!x || !dy || !dx) return GRKAN_ERR_NULL;
+    if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
+    if (overlaps(x, bytes, dx, bytes) || bad_alias(dy, dx, bytes)) return GRKAN_ERR_ALIAS;
+    if (mode == GRKAN_ATOMIC_PER_BLOCK) {
+      const long long sb = block_rows > 0 ? block_rows : 1024;
+      if (((p.rows + sb - 1) / sb) * p.n_g > 0x7fffffffLL) return GRKAN_ERR_SHAPE;
+    }
+  }
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(dA, 0, sizeof(float) * p.n_g * (p.m + 1), st);
   if (e == cudaSuccess && p.n > 0) e = cudaMemsetAsync(dB, 0, sizeof(float) * p.n_g * p.n, st);
   if ((s = cuda_status(e, "grkan_backward_atomic zeroing")) != GRKAN_OK) return s;
   if (p.T == 0) return GRKAN_OK;
-  if (!x || !dy || !dx) return GRKAN_ERR_NULL;
-  if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;
-  const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
-  if (bad_alias(x, dx, bytes) || bad_alias(dy, dx, bytes)) return GRKAN_ERR_ALIAS;
   const bool f32 = p.dtype == GRKAN_F32;
   if (mode == GRKAN_ATOMIC_PER_ELEMENT) {
     const long long elems = p.rows * p.d;
@@ -592,8 +604,7 @@ grkan_status_t grkan_backward_atomic(const void* x, const void* dy, const float*
   } else {
     const int sb = block_rows > 0 ? block_rows : 1024;
     const long long tiles = (p.rows + sb - 1) / sb;
-    const long long blocks = tiles * p.n_g;
-    if (blocks > 0x7fffffffLL) return GRKAN_ERR_SHAPE;
+    const long long blocks = tiles * p.n_g;  // fits in 31 bits (checked above)
     if (f32)
       grk::bwd_atomic_block<grk::IoF32, GRKAN_MAX_M, GRKAN_MAX_N>
           <<<(unsigned)blocks, grk::kAtomicThreads, 0, st>>>(
@@ -891,7 +902,7 @@ grkan_status_t grkan_forward_backward(const void* x, const void* dy, const float
     if (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace))
       return GRKAN_ERR_WORKSPACE;
     const size_t bytes = (size_t)p.rows * (size_t)p.d * (size_t)p.es;
-    if (bad_alias(x, dx, bytes) || bad_alias(dy, dx, bytes) || overlaps(y, bytes, x, bytes) ||
+    if (overlaps(x, bytes, dx, bytes) || bad_alias(dy, dx, bytes) || overlaps(y, bytes, x, bytes) ||
         overlaps(y, bytes, dy, bytes) || overlaps(y, bytes, dx, bytes))
       return GRKAN_ERR_ALIAS;
     if (overlaps(workspace, p.ws_bytes, x, bytes) || overlaps(workspace, p.ws_bytes, dy, bytes) ||
@@ -1059,7 +1070,7 @@ const char* grkan_status_string(grkan_status_t s) {
     case GRKAN_ERR_DTYPE: return "GRKAN_ERR_DTYPE: unknown dtype";
     case GRKAN_ERR_WORKSPACE: return "GRKAN_ERR_WORKSPACE: workspace missing, small or unaligned";
     case GRKAN_ERR_CUDA: return "GRKAN_ERR_CUDA: CUDA error while enqueueing";
-    case GRKAN_ERR_ALIAS: return "GRKAN_ERR_ALIAS: partially overlapping input and output";
+    case GRKAN_ERR_ALIAS: return "GRKAN_ERR_ALIAS: an output overlaps an input it may not overlap";
     case GRKAN_ERR_FLAGS: return "GRKAN_ERR_FLAGS: unknown flag bits";
     case GRKAN_ERR_DEVICE: return "GRKAN_ERR_DEVICE: current device is not sm_100";
   }

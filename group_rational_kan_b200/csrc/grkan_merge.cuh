@@ -2,11 +2,12 @@
 //
 // The first stage leaves one float32 partial per (row tile, group,
 // coefficient). This kernel adds the T partials of each (group, coefficient)
-// in double precision in a fixed order and writes dA / dB. This is the "single
-// controllable merge step" that replaces scattered atomic updates ("PolyKAN:
-// Efficient Fused GPU Operators for Polynomial Kolmogorov-Arnold Network
-// Variants", abstract, technique (iii)); the order never depends on timing,
-// so the result is identical from run to run.
+// in double precision in a fixed order and writes dA / dB: a second-stage
+// merge in a set order takes the place of per-element atomic adds (the
+// two-stage reduction of "PolyKAN: Efficient Fused GPU Operators for
+// Polynomial Kolmogorov-Arnold Network Variants", abstract, technique (iii)).
+// The order never depends on timing, so the result is identical from run to
+// run.
 #pragma once
 
 #include "grkan_common.cuh"

@@ -32,7 +32,12 @@
  * Conventions shared by every entry point:
  *  - Pointers named x, y, dy, dx, a, b, dA, dB, workspace are DEVICE pointers
  *    (or managed memory) of the current CUDA device; the caller owns them.
- *    The library allocates no memory and keeps no per-call state.
+ *    The compute entry points allocate no device memory and keep no state
+ *    between calls; the exceptions are named where they are declared:
+ *    grkan_step_host creates three streams and a few events per device on its
+ *    first call, grkan_backward_noalloc uses a static device array that the
+ *    library holds, and the fused linear entry points look up a per-device
+ *    occupancy figure once.
  *  - dtype selects the element type of x, y, dy, dx: float32 or bfloat16.
  *    Coefficients a (n_g x (m+1)), b (n_g x n) and gradients dA, dB are always
  *    float32, row-major. Arithmetic is float32; the merge is float64.
@@ -41,8 +46,10 @@
  *  - 0 <= m <= GRKAN_MAX_M, 0 <= n <= GRKAN_MAX_N, n_g >= 1, d % n_g == 0.
  *    With n = 0, b may be NULL and Q = 0. B*N*d == 0 is a valid no-op
  *    (the backward then writes zeros to dA and dB).
- *  - Aliasing: y may equal x (in place) and dx may equal dy or x; any other
- *    overlap between an input and an output returns GRKAN_ERR_ALIAS.
+ *  - Aliasing: y may equal x (in place) and dx may equal dy (dy is read
+ *    before dx is written at the same place). dx may not equal or overlap x,
+ *    which has to stay readable for the caller; that, and any other overlap
+ *    between an input and an output, returns GRKAN_ERR_ALIAS.
  *  - Errors are returned, never thrown; on error nothing is enqueued.
  *    GRKAN_ERR_CUDA reports a launch failure (cudaGetLastError); a fault that
  *    happens later on the GPU surfaces at the caller's next synchronisation.
@@ -77,7 +84,7 @@ typedef enum grkan_status {
   GRKAN_ERR_DTYPE = 4,     /* unknown dtype */
   GRKAN_ERR_WORKSPACE = 5, /* workspace NULL or smaller than the query says */
   GRKAN_ERR_CUDA = 6,      /* CUDA reported an error while enqueueing */
-  GRKAN_ERR_ALIAS = 7,     /* partially overlapping input and output */
+  GRKAN_ERR_ALIAS = 7,     /* an output overlaps an input it may not overlap */
   GRKAN_ERR_FLAGS = 8,     /* unknown flag bits */
   GRKAN_ERR_DEVICE = 9     /* the current device is not sm_100 (B200 class) */
 } grkan_status_t;

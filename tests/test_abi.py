@@ -95,22 +95,46 @@ def test_argument_errors_need_no_gpu():
 
 
 def test_backward_argument_errors_need_no_gpu():
-    A = 1 << 20
-    W = 1 << 30
+    X = 1 << 20   # x and dy (inputs may share memory)
+    D = 1 << 24   # dx
+    W = 1 << 30   # workspace
     shape = (2, 3, 12, 3, 5, 4, grk.F32)
+    nbytes = 2 * 3 * 12 * 4
     need = grk.grkan_backward_workspace_bytes(*shape)
     assert need > 0
     b = grk.grkan_backward_ex
-    assert b(A, A, A, A, A, None, A, *shape, W, need, 0, 0) == NULL
-    assert b(A, A, A, A, A, A, None, *shape, W, need, 0, 0) == NULL
-    assert b(A, A, A, A, A, A, A, *shape, None, need, 0, 0) == WORKSPACE
-    assert b(A, A, A, A, A, A, A, *shape, W, need - 4, 0, 0) == WORKSPACE
-    assert b(A, A, A, A, A, A, A, *shape, W + 4, need, 0, 0) == WORKSPACE  # unaligned
-    assert b(A, A, A, A, A + 8, A, A, *shape, W, need, 0, 0) == ALIAS
-    assert b(A, A, A, A, A, A, A, *shape, A + 16, need, 0, 0) == ALIAS  # workspace inside x
-    assert b(A, A, A, A, A, A, A, *shape, W, need, 4, 0) == FLAGS
+    assert b(X, X, X, X, D, None, X, *shape, W, need, 0, 0) == NULL
+    assert b(X, X, X, X, D, X, None, *shape, W, need, 0, 0) == NULL
+    assert b(X, X, X, X, D, X, X, *shape, None, need, 0, 0) == WORKSPACE
+    assert b(X, X, X, X, D, X, X, *shape, W, need - 4, 0, 0) == WORKSPACE
+    assert b(X, X, X, X, D, X, X, *shape, W + 4, need, 0, 0) == WORKSPACE  # unaligned
+    assert b(X, X, X, X, X + 8, X, X, *shape, W, need, 0, 0) == ALIAS  # dx overlaps x
+    assert b(X, X, X, X, X, X, X, *shape, W, need, 0, 0) == ALIAS  # dx == x: x must stay
+    assert b(X, D + 16, X, X, D, X, X, *shape, W, need, 0, 0) == ALIAS  # dx overlaps dy
+    assert b(X, X, X, X, D, X, X, *shape, X + 16, need, 0, 0) == ALIAS  # workspace inside x
+    assert b(X, X, X, X, D, X, X, *shape, D + nbytes - 16, need, 0, 0) == ALIAS  # ... inside dx
+    assert b(X, X, X, X, D, X, X, *shape, W, need, 4, 0) == FLAGS
+    fb = grk.grkan_forward_backward
+    Y = 1 << 28
+    assert fb(X, D, X, X, Y, X, X, X, *shape, W, need, 0, 0) == ALIAS  # dx == x
+    assert fb(X, D, X, X, X, D, X, X, *shape, W, need, 0, 0) == ALIAS  # y == x
+    at = grk.grkan_backward_atomic
+    assert at(X, X, X, X, X, X, X, *shape, 1, 0, 0) == ALIAS  # dx == x
     if not _has_gpu():
-        assert b(A, A, A, A, A, A, A, *shape, W, need, 0, 0) == DEVICE
+        assert b(X, X, X, X, D, X, X, *shape, W, need, 0, 0) == DEVICE
+        assert b(X, D, X, X, D, X, X, *shape, W, need, 0, 0) == DEVICE  # dx == dy is allowed
+        assert fb(X, D, X, X, Y, D, X, X, *shape, W, need, 0, 0) == DEVICE
+
+
+def test_huge_rows_of_narrow_groups_take_the_generic_path():
+    """The pipelined kernels keep a lane's offsets inside a TMA box in 32-bit
+    integers; shapes whose box would span 2^31 bytes or more go to the generic
+    kernels (bf16, d_g = 8: 192-row backward boxes)."""
+    A = 1 << 20
+    assert grk.grkan_forward_path(A, A, 1, 1, 8 << 10, 1 << 10, 5, 4, grk.BF16) == 1
+    assert grk.grkan_backward_path(A, A, A, 1, 1, 8 << 10, 1 << 10, 5, 4, grk.BF16) == 1
+    assert grk.grkan_forward_path(A, A, 1, 1, 8 << 20, 1 << 20, 5, 4, grk.BF16) == 0
+    assert grk.grkan_backward_path(A, A, A, 1, 1, 8 << 20, 1 << 20, 5, 4, grk.BF16) == 0
 
 
 def _has_gpu():

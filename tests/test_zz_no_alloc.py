@@ -16,7 +16,6 @@ import synth
 
 pytestmark = pytest.mark.gpu
 
-RTOL = {synth.F32: 1e-5, synth.BF16: 1e-2}
 
 
 def _inputs(w):
@@ -45,13 +44,12 @@ def _via_noalloc(w, tx, tdy, ta, tb):
     return dx, dA, dB
 
 
-def _same(w, got, ref):
-    dx, dA, dB = got
-    rdx, rdA, rdB = ref
-    rt = RTOL[w.dtype]
-    assert torch.all((dx.double() - rdx.double()).abs() <= rt * rdx.double().abs())
-    assert torch.all((dA.double() - rdA.double()).abs() <= 1e-4 * rdA.double().abs())
-    assert torch.all((dB.double() - rdB.double()).abs() <= 1e-4 * rdB.double().abs())
+def _same(got, ref):
+    # the same plan, kernels, partial layout and merge order as grkan_backward:
+    # the results must be the same bits (a leftover partial from an earlier call
+    # or a skipped tile would show up here, however small)
+    for u, v in zip(got, ref):
+        assert torch.equal(u, v)
 
 
 def test_noalloc_matches_workspace_entry_point_call_after_call():
@@ -63,7 +61,7 @@ def test_noalloc_matches_workspace_entry_point_call_after_call():
     # must not leak into the next result
     for _ in range(2):
         for p, ref in zip(prepared, refs):
-            _same(p[0], _via_noalloc(*p), ref)
+            _same(_via_noalloc(*p), ref)
     st, code = grk.grkan_device_error()
     assert st == 0 and code == 0
 
