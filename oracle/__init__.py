@@ -9,7 +9,14 @@ Pins (checked by ``tests/test_oracle_*.py`` against things other than the
 oracle itself): identity initialisation, the b = 0 polynomial special case,
 exact rational brute force on dyadic inputs, central finite differences for dx,
 dA and dB, x = 0, linearity in dy, group relabelling, and an fp64 autograd
-witness. Every function here is pinned.
+witness. The error scales that set the y / dx tolerances are pinned too:
+kappa_q by brute force over the sign patterns of b, kappa_y as the largest
+first-order sensitivity of y to relative coefficient perturbations (exact dual
+numbers over every sign pattern) and by a closed form at nonnegative inputs,
+kappa_dx by a closed form at nonnegative inputs, sign invariances and the
+perturbation bound it gives, and the c2 noise scales by closed forms. Every
+function here is pinned; ``tests/test_oracle_mutants.py`` plants 36 mistakes
+and each one trips a pin.
 """
 import ctypes
 import os

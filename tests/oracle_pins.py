@@ -16,6 +16,19 @@ What pins what:
          L = sum dy y (exact: L is linear in a), brute force, linearity in dy
   dB     b = 0 gives 0, central differences (Richardson), brute force,
          autograd witness, group relabelling
+  error scales (which widen every y / dx comparison and pick the elements
+  whose sign of Q is undecidable in float32):
+         kappa_q  = max over the 2^n sign patterns of b of |Q| (brute force)
+         kappa_y  = the largest first-order change of y under relative
+                    coefficient perturbations of size one, over every sign
+                    pattern (exact dual numbers); closed form (P + yQ) / D at
+                    nonnegative x, a, b (exact rationals)
+         kappa_dx = closed form at nonnegative x, a, b, dy (exact rationals);
+                    invariant under a -> -a, b -> -b, dy -> -dy; bounds the
+                    first-order change of dx under relative coefficient
+                    perturbations (with the |dx| kappa_q / D part that the
+                    relative tolerance term covers)
+         c2       = closed forms at nonnegative inputs with b != 0
 """
 from fractions import Fraction
 
@@ -390,7 +403,233 @@ def pin_library_polyval(orc):
             assert np.all(yg[eq] == np.abs(P[eq])), "|y| = |P| where Q = 0"
 
 
+# --- error scales -------------------------------------------------------------
+#
+# kappa_y, kappa_dx and kappa_q widen the y / dx tolerances and decide which
+# elements count as sign-ambiguous, so an inflated scale would silently loosen
+# every parity check. They are pinned here to what they mean, not to their
+# formulas.
+
+def _fpoly(coefs, x):
+    """sum_k coefs[k] x^k over Fractions (plain power sum)."""
+    return sum((c * x ** k for k, c in enumerate(coefs)), Fraction(0))
+
+
+def _nonneg_case(rng, rows, d, n_g, m, n):
+    x = _dyadic(rng, (rows, d), 8, 24)
+    x = np.abs(x)
+    x[0, 0] = 0.0
+    dy = np.abs(_dyadic(rng, (rows, d), 8, 16))
+    a = np.abs(_dyadic(rng, (n_g, m + 1), 8, 8))
+    b = np.abs(_dyadic(rng, (n_g, n), 8, 8))
+    b[:, 0] = np.maximum(b[:, 0], 0.125)  # Q > 0 wherever x > 0
+    return x, dy, a, b
+
+
+def _pqs(xv, ga, gb):
+    """Exact P, P', Q, Q' at a Fraction x for group coefficients (floats)."""
+    fa = [Fraction(float(v)) for v in ga]
+    fb = [Fraction(0)] + [Fraction(float(v)) for v in gb]  # Q has no constant term
+    P = _fpoly(fa, xv)
+    Q = _fpoly(fb, xv)
+    dP = _fpoly([k * c for k, c in enumerate(fa)][1:], xv)
+    dQ = _fpoly([k * c for k, c in enumerate(fb)][1:], xv)
+    return P, dP, Q, dQ
+
+
+def pin_kappa_q_brute_force(orc):
+    """kappa_q = sum_j |b_j||x|^j is the largest |Q(x)| over the 2^n sign
+    patterns of (b_1..b_n) (numpy's polynomial evaluator), the scale that
+    float32 rounding of Q is measured against."""
+    from numpy.polynomial import polynomial as npp
+    import itertools
+    rng = np.random.default_rng(31)
+    for (m, n) in ((5, 4), (2, 6), (3, 1)):
+        rows, d, n_g = 5, 8, 2
+        x, dy, a, b = _rand_case(rng, rows, d, n_g, m, n, xs=1.5, coef=0.8)
+        x[0, 0] = 0.0
+        _, ex = orc.backward_elem(x, dy, a, b, n_g, extras=True)
+        dg = d // n_g
+        for g in range(n_g):
+            xs = x[:, g * dg:(g + 1) * dg].astype(np.float64)
+            best = np.zeros_like(xs)
+            for signs in itertools.product((-1.0, 1.0), repeat=n):
+                cb = np.concatenate([[0.0], np.abs(b[g].astype(np.float64)) * signs])
+                best = np.maximum(best, np.abs(npp.polyval(xs, cb)))
+            _close(ex["kappa_q"][:, g * dg:(g + 1) * dg], best, 1e-14, 1e-300,
+                   "kappa_q (m=%d n=%d)" % (m, n))
+
+
+def pin_kappa_y_nonneg_closed_form(orc):
+    """With x, a, b >= 0 every term is nonnegative, so the absolute-value
+    evaluation is the evaluation itself: kappa_y = (P + y Q) / D
+    = P (1 + 2Q) / (1 + Q)^2, in exact rationals."""
+    rng = np.random.default_rng(32)
+    for (m, n, n_g, d) in ((5, 4, 2, 8), (3, 3, 1, 4), (7, 2, 2, 4)):
+        x, dy, a, b = _nonneg_case(rng, 3, d, n_g, m, n)
+        _, ky = orc.forward(x, a, b, n_g, kappa=True)
+        dg = d // n_g
+        for r in range(x.shape[0]):
+            for c in range(d):
+                P, _, Q, _ = _pqs(Fraction(float(x[r, c])), a[c // dg], b[c // dg])
+                want = P * (1 + 2 * Q) / (1 + Q) ** 2
+                assert abs(Fraction(float(ky[r, c])) - want) <= Fraction(1, 10 ** 13) * want, \
+                    "kappa_y closed form at (%d,%d), m=%d n=%d" % (r, c, m, n)
+
+
+def pin_kappa_y_max_sensitivity(orc):
+    """kappa_y is the largest first-order change of y when every coefficient
+    takes a relative perturbation of size one (a_i -> a_i (1 + t s_i),
+    b_j -> b_j (1 + t r_j), s, r = +-1): brute force over all 2^(m+1+n) sign
+    patterns with exact dual numbers, at points with Q != 0 and both signs of
+    x, y and the coefficients."""
+    import itertools
+    rng = np.random.default_rng(33)
+    for (m, n, cnt) in ((3, 2, 10), (5, 4, 4)):
+        x = _dyadic(rng, (cnt,), 8, 24)
+        x[x == 0] = 0.625
+        a = _dyadic(rng, (m + 1,), 8, 8)
+        b = _dyadic(rng, (n,), 8, 8)
+        b[0] = 0.375 if b[0] == 0 else b[0]
+        _, ky = orc.forward(x.reshape(1, -1), a.reshape(1, -1), b.reshape(1, -1), 1, kappa=True)
+        fa = [Fraction(float(v)) for v in a]
+        fb = [Fraction(float(v)) for v in b]
+        seen_neg_y = False
+        for e in range(cnt):
+            xv = exact.Dual(Fraction(float(x[e])))
+            if exact.activation(xv, fa, fb).v < 0:
+                seen_neg_y = True
+            best = Fraction(0)
+            for signs in itertools.product((-1, 1), repeat=m + 1 + n):
+                aa = [exact.Dual(v, signs[i] * v) for i, v in enumerate(fa)]
+                bb = [exact.Dual(v, signs[m + 1 + j] * v) for j, v in enumerate(fb)]
+                out = exact.activation(xv, aa, bb)
+                best = max(best, abs(out.d))
+            assert abs(Fraction(float(ky[0, e])) - best) <= Fraction(1, 10 ** 13) * best, \
+                "kappa_y vs max sensitivity at x=%g (m=%d n=%d): %r vs %r" % (
+                    float(x[e]), m, n, float(ky[0, e]), float(best))
+        assert seen_neg_y
+
+
+def pin_kappa_dx_nonneg_closed_form(orc):
+    """With x, a, b, dy >= 0 (so Q >= 0, s = 1 where x > 0): kappa_dx
+    = dy (P' + y Q' + kappa_y Q') / D = dy (P' + Q' P (2 + 3Q) / (1 + Q)^2) / (1 + Q),
+    in exact rationals."""
+    rng = np.random.default_rng(34)
+    for (m, n, n_g, d) in ((5, 4, 2, 8), (3, 3, 1, 4), (7, 2, 2, 4)):
+        x, dy, a, b = _nonneg_case(rng, 3, d, n_g, m, n)
+        _, ex = orc.backward_elem(x, dy, a, b, n_g, extras=True)
+        dg = d // n_g
+        for r in range(x.shape[0]):
+            for c in range(d):
+                P, dP, Q, dQ = _pqs(Fraction(float(x[r, c])), a[c // dg], b[c // dg])
+                g = Fraction(float(dy[r, c]))
+                want = g * (dP + dQ * P * (2 + 3 * Q) / (1 + Q) ** 2) / (1 + Q)
+                got = Fraction(float(ex["kappa_dx"][r, c]))
+                assert abs(got - want) <= Fraction(1, 10 ** 13) * want, \
+                    "kappa_dx closed form at (%d,%d), m=%d n=%d: %r vs %r" % (
+                        r, c, m, n, float(got), float(want))
+
+
+def pin_kappa_dx_sign_invariance(orc):
+    """kappa_dx is a sum of absolute values: negating every a_i (which negates
+    P, P', y), every b_j (which negates Q, Q') or dy leaves it unchanged bit for
+    bit."""
+    rng = np.random.default_rng(35)
+    rows, d, n_g, m, n = 6, 12, 3, 5, 4
+    x, dy, a, b = _rand_case(rng, rows, d, n_g, m, n, xs=1.5)
+    x[0, :2] = 0.0
+    base = orc.backward_elem(x, dy, a, b, n_g, extras=True)[1]
+    for what, args in (("-a", (x, dy, -a, b)), ("-b", (x, dy, a, -b)), ("-dy", (x, -dy, a, b))):
+        ex = orc.backward_elem(*args, n_g, extras=True)[1]
+        assert np.array_equal(ex["kappa_dx"], base["kappa_dx"]), "kappa_dx changes under " + what
+        assert np.array_equal(ex["kappa_q"], base["kappa_q"]), "kappa_q changes under " + what
+    _, ky0 = orc.forward(x, a, b, n_g, kappa=True)
+    for aa, bb in ((-a, b), (a, -b)):
+        assert np.array_equal(orc.forward(x, aa, bb, n_g, kappa=True)[1], ky0), "kappa_y sign"
+
+
+def pin_kappa_dx_bounds_perturbation(orc):
+    """Relative coefficient perturbations of size eta change dx by at most
+    eta (kappa_dx + |dx| kappa_q / D) to first order (the second part is the
+    effect of D's error on the 1/D factor, covered by the relative part of the
+    tolerance), and over the elements the largest change seen under random
+    sign patterns reaches that bound (an inflated kappa_dx fails there)."""
+    rng = np.random.default_rng(36)
+    rows, d, n_g, m, n = 6, 16, 2, 5, 4
+    x, dy, a, b = _rand_case(rng, rows, d, n_g, m, n, xs=1.5, coef=0.7)
+    dx, ex = orc.backward_elem(x, dy, a, b, n_g, extras=True)
+    q = ex["q"]
+    Dv = 1.0 + np.abs(q)
+    bound = ex["kappa_dx"] + np.abs(dx) * ex["kappa_q"] / Dv
+    eta = 2.0 ** -26
+    a64, b64 = a.astype(np.float64), b.astype(np.float64)
+    reach = np.zeros_like(dx)
+    for _ in range(48):
+        sa = rng.choice([-1.0, 1.0], a.shape)
+        sb = rng.choice([-1.0, 1.0], b.shape)
+        # the oracle widens float32 coefficients exactly; feed it the perturbed
+        # values through its double-precision arrays
+        o_p = _backward_f64(orc, x, dy, a64 * (1 + eta * sa), b64 * (1 + eta * sb), n_g)
+        o_m = _backward_f64(orc, x, dy, a64 * (1 - eta * sa), b64 * (1 - eta * sb), n_g)
+        change = np.abs(o_p - o_m) / (2 * eta)
+        smooth = np.abs(q) > 1e-6
+        assert np.all(change[smooth] <= bound[smooth] * (1 + 1e-5) + 1e-12), "dx moves beyond kappa"
+        reach = np.maximum(reach, change)
+    # No element-wise lower bound exists (one coefficient moves P' and y in
+    # ways that can cancel), but over the elements the bound is reached and
+    # typically nearly so: an inflated kappa_dx fails both.
+    sm = np.abs(q) > 1e-6
+    assert np.max(reach[sm] / bound[sm]) >= 0.95, "no element reaches the bound"
+    assert np.median(reach[sm] / ex["kappa_dx"][sm]) >= 0.6, "kappa_dx far above dx's sensitivity"
+
+
+def _backward_f64(orc, x, dy, a64, b64, n_g):
+    """dx with float64 coefficients (bypassing the float32 widening)."""
+    rows, d = x.shape
+    m = a64.shape[1] - 1
+    n = b64.shape[1]
+    out = np.empty(rows * d, np.float64)
+    a64 = np.ascontiguousarray(a64)
+    b64 = np.ascontiguousarray(b64)
+    rc = orc.lib.gro_backward_elem(x.ctypes.data, np.ascontiguousarray(dy).ctypes.data, 0, rows,
+                                   d, n_g, m, n, a64.ctypes.data, b64.ctypes.data, None,
+                                   rows * d, out.ctypes.data, None, None, None, None)
+    assert rc == 0
+    return out.reshape(rows, d)
+
+
+def pin_noise_scales_nonneg(orc):
+    """c2 with b != 0, at x, a, b, dy >= 0 (Q >= 0, s = 1 where x > 0): the dA
+    weight is |t x^i| (1 + Q/D) = dy x^i (1 + 2Q) / (1 + Q)^2 and the dB weight
+    |t y x^j| + |dy x^j / D^2| (P + 2 P Q / D) = 2 dy x^j P (1 + 2Q) / (1 + Q)^3,
+    summed in squares over the group (exact rationals)."""
+    rng = np.random.default_rng(37)
+    rows, d, n_g, m, n = 4, 8, 2, 5, 4
+    x, dy, a, b = _nonneg_case(rng, rows, d, n_g, m, n)
+    x[x == 0] = 0.25  # s = 1 everywhere
+    g = orc.coef_grads(x, dy, a, b, n_g)
+    dg = d // n_g
+    for gi in range(n_g):
+        wa = [Fraction(0)] * (m + 1)
+        wb = [Fraction(0)] * n
+        for r in range(rows):
+            for c in range(gi * dg, (gi + 1) * dg):
+                xv = Fraction(float(x[r, c]))
+                gv = Fraction(float(dy[r, c]))
+                P, _, Q, _ = _pqs(xv, a[gi], b[gi])
+                for i in range(m + 1):
+                    wa[i] += (gv * xv ** i * (1 + 2 * Q) / (1 + Q) ** 2) ** 2
+                for j in range(1, n + 1):
+                    wb[j - 1] += (2 * gv * xv ** j * P * (1 + 2 * Q) / (1 + Q) ** 3) ** 2
+        _close(g["c2_a"][gi], [float(v) for v in wa], 1e-13, 0, "c2_a nonneg")
+        _close(g["c2_b"][gi], [float(v) for v in wb], 1e-13, 0, "c2_b nonneg")
+
+
 ALL_PINS = [pin_identity, pin_polynomial_b0, pin_dyadic_exact, pin_x_zero, pin_bf16_widening,
             pin_fd_dx, pin_fd_dA, pin_fd_dB, pin_autograd, pin_linearity, pin_group_relabel,
             pin_thread_invariance, pin_sampled_and_extras, pin_ambiguity, pin_noise_scales,
-            pin_library_polyval]
+            pin_library_polyval, pin_kappa_q_brute_force, pin_kappa_y_nonneg_closed_form,
+            pin_kappa_y_max_sensitivity, pin_kappa_dx_nonneg_closed_form,
+            pin_kappa_dx_sign_invariance, pin_kappa_dx_bounds_perturbation,
+            pin_noise_scales_nonneg]

@@ -45,6 +45,37 @@ MUTANTS = [
      0),
     ("forward groups interleaved", "int g = (int)((e % d) / dg);",
      "int g = (int)((e % d) % n_g);", 0),
+    # the error scales that widen the y / dx tolerances and the sign-ambiguity test
+    ("kappa_y drops the denominator term", "return (sa + fabs(p->y) * sb) / p->D;",
+     "return sa / p->D;", 0),
+    ("kappa_y misses the 1/D", "return (sa + fabs(p->y) * sb) / p->D;",
+     "return sa + fabs(p->y) * sb;", 0),
+    ("kappa_y uses the signed y", "return (sa + fabs(p->y) * sb) / p->D;",
+     "return (sa + p->y * sb) / p->D;", 0),
+    ("kappa_y doubled", "return (sa + fabs(p->y) * sb) / p->D;",
+     "return 2.0 * (sa + fabs(p->y) * sb) / p->D;", 0),
+    ("kappa_y denominator powers start at x^0", "  xi = ax;\n  for (int j = 1; j <= n; ++j) {",
+     "  xi = 1.0;\n  for (int j = 1; j <= n; ++j) {", 0),
+    ("kappa_q powers start at x^0", "double ax = fabs(x), sb = 0.0, xi = ax;",
+     "double ax = fabs(x), sb = 0.0, xi = 1.0;", 0),
+    ("kappa_q uses the signed x", "double ax = fabs(x), sb = 0.0, xi = ax;",
+     "double ax = x, sb = 0.0, xi = ax;", 0),
+    ("kappa_q doubled", "  return sb;\n}", "  return 2.0 * sb;\n}", 0),
+    ("kappa_dx drops the kappa_y |Q'| term",
+     "(sa + fabs(p.y) * sb + ky * fabs(p.dQ)) / p.D;", "(sa + fabs(p.y) * sb) / p.D;", 0),
+    ("kappa_dx misses the 1/D", "(sa + fabs(p.y) * sb + ky * fabs(p.dQ)) / p.D;",
+     "(sa + fabs(p.y) * sb + ky * fabs(p.dQ));", 0),
+    ("kappa_dx doubled", "kappa_dx[k] = fabs(gv) * (", "kappa_dx[k] = 2.0 * fabs(gv) * (", 0),
+    ("kappa_dx drops the factor i", "sa += (double)i * fabs(ga[i]) * xi;",
+     "sa += fabs(ga[i]) * xi;", 0),
+    ("kappa_dx uses the signed y", "(sa + fabs(p.y) * sb + ky * fabs(p.dQ)) / p.D;",
+     "(sa + p.y * sb + ky * fabs(p.dQ)) / p.D;", 0),
+    ("kappa_dx uses the signed Q'", "(sa + fabs(p.y) * sb + ky * fabs(p.dQ)) / p.D;",
+     "(sa + fabs(p.y) * sb + ky * p.dQ) / p.D;", 0),
+    ("dA noise weight drops kappa_q / D", "double w = fabs(term) * (1.0 + kq / p.D);",
+     "double w = fabs(term);", 0),
+    ("dB noise weight drops the 2|P| kappa_q / D part", "(kp + 2.0 * fabs(p.P) * kq / p.D)",
+     "(kp)", 0),
 ]
 
 
