@@ -415,14 +415,16 @@ def main():
     scratch = torch.empty(sneed, dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        check(grk.grkan_step_host(x_h, dy_h, a, b, y_h, dx_h, dA_h, dB_h, B, N, d, n_g, m, n, dt,
-                                  scratch, sneed, 0, sp), "step_host")
-        if world > 1:  # the data-parallel exchange of this rank's gradients
-            stream.synchronize()
-            s64 = torch.from_numpy(np.concatenate([dA_h.numpy(), dB_h.numpy()], 1)).to(
-                dev, torch.float64)
-            g = all_gather_sums(s64)
+        # at N > 1 the step also leaves this rank's float64 sums on the device; the
+        # ranks exchange them and merge in rank order, then the gradients go to
+        # the host (the same bits on every rank)
+        check(grk.grkan_step_host(x_h, dy_h, a, b, y_h, dx_h, dA_h, dB_h, sums64, B, N, d, n_g,
+                                  m, n, dt, scratch, sneed, 0, sp), "step_host")
+        if world > 1:
+            g = all_gather_sums(sums64)
             check(grk.grkan_merge_ranks(g, world, dA, dB, n_g, m, n, sp), "merge_ranks")
+            dA_h.copy_(dA, non_blocking=True)
+            dB_h.copy_(dB, non_blocking=True)
 
     for _ in range(min(2, args.e2e_steps)):
         e2e_step()

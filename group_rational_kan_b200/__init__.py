@@ -31,7 +31,7 @@ F32, BF16 = 0, 1
 FLAG_GENERIC = 1
 NOALLOC_WORKSPACE_BYTES = 4 << 20  # GRKAN_NOALLOC_WORKSPACE_BYTES
 DEVICE_ERROR_SELFTEST = 16  # GRKAN_DEVICE_ERROR_SELFTEST
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libgrkan_b200.so")
@@ -82,7 +82,7 @@ def _load():
         "grkan_forward_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                        ctypes.c_int, P, SZ, U32, P]),
         "grkan_step_host_scratch_bytes": (SZ, [I64, I64, I64, I32, I32, I32, ctypes.c_int, I64]),
-        "grkan_step_host": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
+        "grkan_step_host": (S, [P, P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                 ctypes.c_int, P, SZ, I64, P]),
         "grkan_backward_noalloc": (S, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32,
                                        ctypes.c_int, P]),
@@ -260,13 +260,15 @@ def grkan_step_host_scratch_bytes(B, N, d, n_g, m, n, dtype, chunk_rows=0):
     return lib().grkan_step_host_scratch_bytes(B, N, d, n_g, m, n, dtype, chunk_rows)
 
 
-def grkan_step_host(x_host, dy_host, a, b, y_host, dx_host, dA_host, dB_host, B, N, d, n_g, m, n,
-                    dtype, scratch, scratch_bytes, chunk_rows=0, stream=None):
+def grkan_step_host(x_host, dy_host, a, b, y_host, dx_host, dA_host, dB_host, sums64, B, N, d,
+                    n_g, m, n, dtype, scratch, scratch_bytes, chunk_rows=0, stream=None):
     """Forward + backward of host tensors (pinned torch CPU tensors or raw host
-    pointers) streamed through device scratch; dA_host / dB_host are host."""
+    pointers) streamed through device scratch; dA_host / dB_host are host,
+    sums64 (float64 sums for a data-parallel merge) is a device tensor or None."""
     return lib().grkan_step_host(_ptr(x_host), _ptr(dy_host), _ptr(a), _ptr(b), _ptr(y_host),
-                                 _ptr(dx_host), _ptr(dA_host), _ptr(dB_host), B, N, d, n_g, m, n,
-                                 dtype, _ptr(scratch), scratch_bytes, chunk_rows, _stream(stream))
+                                 _ptr(dx_host), _ptr(dA_host), _ptr(dB_host), _ptr(sums64), B, N,
+                                 d, n_g, m, n, dtype, _ptr(scratch), scratch_bytes, chunk_rows,
+                                 _stream(stream))
 
 
 def grkan_forward_path(x, y, B, N, d, n_g, m, n, dtype, flags=0):

@@ -924,8 +924,8 @@ size_t grkan_step_host_scratch_bytes(int64_t B, int64_t N, int64_t d, int32_t n_
 
 grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const float* a,
                                const float* b, void* y_host, void* dx_host, float* dA_host,
-                               float* dB_host, int64_t B, int64_t N, int64_t d, int32_t n_g,
-                               int32_t m, int32_t n, grkan_dtype_t dtype, void* scratch,
+                               float* dB_host, double* sums64, int64_t B, int64_t N, int64_t d,
+                               int32_t n_g, int32_t m, int32_t n, grkan_dtype_t dtype, void* scratch,
                                size_t scratch_bytes, int64_t chunk_rows, void* stream) {
   Plan p;
   grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
@@ -963,7 +963,7 @@ grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const fl
   GRK_TRY(cudaStreamWaitEvent(hp->s_comp, hp->start, 0), "cudaStreamWaitEvent");
   GRK_TRY(cudaStreamWaitEvent(hp->s_out, hp->start, 0), "cudaStreamWaitEvent");
   if (empty) {
-    s = do_merge(p, ws, 0, dA, dB, nullptr, hp->s_comp);
+    s = do_merge(p, ws, 0, dA, dB, sums64, hp->s_comp);
     if (s != GRKAN_OK) return s;
   } else {
     const long long nchunks = (p.rows + L.chunk_rows - 1) / L.chunk_rows;
@@ -1009,7 +1009,7 @@ grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const fl
                               hp->s_out), "cudaMemcpyAsync");
       GRK_TRY(cudaEventRecord(hp->out[slot], hp->s_out), "cudaEventRecord");
     }
-    s = do_merge(p, ws, p.ws_bytes, dA, dB, nullptr, hp->s_comp);
+    s = do_merge(p, ws, p.ws_bytes, dA, dB, sums64, hp->s_comp);
     if (s != GRKAN_OK) return s;
   }
   GRK_TRY(cudaMemcpyAsync(dA_host, dA, ka, cudaMemcpyDeviceToHost, hp->s_comp), "cudaMemcpyAsync");

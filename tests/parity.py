@@ -76,6 +76,16 @@ def check_dx(got, ref, ex, rtol, what="dx"):
 def check_coef(dA, dB, ref, rtol=RTOL_COEF, floor=2e-6, what=""):
     """dA, dB: numpy arrays from the GPU; ref: oracle.coef_grads dict. Returns
     the largest plain relative error (for information)."""
+    return coef_report(dA, dB, ref, rtol, floor, what)["max_rel"]
+
+
+def coef_report(dA, dB, ref, rtol=RTOL_COEF, floor=2e-6, what="", plain=False):
+    """Checks dA, dB as check_coef does and returns a summary: the largest plain
+    relative error over all entries, the largest over the graded entries
+    (|ref| >= 1e-8 sum |term|; sums that cancel below that are reported, not
+    graded), and how many entries pass only through the noise floor or the
+    sign-ambiguity allowance. With plain=True every graded entry must also meet
+    the plain |gpu - ref| <= rtol |ref|."""
     dA = np.asarray(dA, np.float64)
     dB = np.asarray(dB, np.float64)
     eA = np.abs(dA - ref["dA"])
@@ -88,4 +98,19 @@ def check_coef(dA, dB, ref, rtol=RTOL_COEF, floor=2e-6, what=""):
                                                          np.argwhere(~okA)[:4].tolist())
     assert okB.all(), "%s dB: max rel err %.3g at %s" % (what, float(relB.max()),
                                                          np.argwhere(~okB)[:4].tolist())
-    return max(float(relA.max(initial=0)), float(relB.max(initial=0)))
+    gA = np.abs(ref["dA"]) >= 1e-8 * ref["sabs_a"]
+    gB = np.abs(ref["dB"]) >= 1e-8 * ref["sabs_b"]
+    plainA = eA <= rtol * np.abs(ref["dA"])
+    plainB = eB <= rtol * np.abs(ref["dB"])
+    rep = {
+        "max_rel": max(float(relA.max(initial=0)), float(relB.max(initial=0))),
+        "max_rel_graded": max(float(relA[gA].max(initial=0)), float(relB[gB].max(initial=0))),
+        "entries": int(relA.size + relB.size),
+        "ungraded": int((~gA).sum() + (~gB).sum()),
+        "floor_only": int((okA & ~plainA).sum() + (okB & ~plainB).sum()),
+    }
+    if plain:
+        assert np.all(plainA[gA]) and np.all(plainB[gB]), \
+            "%s: plain %.0e relative fails on graded entries (max %.3g)" % (
+                what, rtol, rep["max_rel_graded"])
+    return rep

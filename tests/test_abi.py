@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(grk.library_path if os.path.exists(grk.library_path) else grk.lib()._name)
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert grk.grkan_abi_version() == 1
+    assert grk.grkan_abi_version() == grk.ABI_VERSION == 2
 
 
 def test_status_strings():

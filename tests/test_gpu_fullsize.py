@@ -9,7 +9,7 @@ import torch
 import group_rational_kan_b200 as grk
 import oracle
 import synth
-from parity import RTOL, check_coef, check_dx, check_y, to_f64, to_torch
+from parity import RTOL, check_dx, check_y, coef_report, to_f64, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -53,9 +53,15 @@ def test_fullsize(name, n_g):
     check_dx(dx_s, dx_ref, ex, rtol, "%s dx" % w.name)
 
     g_ref = oracle.coef_grads(x, dy, a, b, w.n_g)
-    rel = check_coef(dA.cpu().numpy(), dB.cpu().numpy(), g_ref, what=w.name)
-    print("%s: max plain relative error of dA/dB %.3g, ambiguous signs %d" % (
-        w.name, rel, g_ref["amb_count"]))
+    # The KAT-shaped workloads meet the plain 1e-4 relative bound on every entry
+    # whose sum does not cancel below 1e-8 of its terms' magnitudes; the noise
+    # floor is needed only for the heavy-tailed stress sweep.
+    rep = coef_report(dA.cpu().numpy(), dB.cpu().numpy(), g_ref, what=w.name,
+                      plain=name != "stress")
+    print("%s: dA/dB max plain relative error %.3g (graded entries %.3g), %d of %d entries "
+          "pass only through the noise floor or the sign allowance, %d ungraded; ambiguous "
+          "signs %d" % (w.name, rep["max_rel"], rep["max_rel_graded"], rep["floor_only"],
+                        rep["entries"], rep["ungraded"], g_ref["amb_count"]))
 
     for _ in range(2):
         again = grk.backward(tx, tdy, ta, tb, w.n_g)

@@ -35,8 +35,9 @@ def test_host_step_matches_device_calls(name, rows, chunk):
     scratch = torch.empty(need, dtype=torch.uint8, device="cuda")
     s = torch.cuda.Stream()
     for _ in range(2):  # a second call reuses streams, events and staging slots
-        st = grk.grkan_step_host(xh, dyh, a, b, yh, dxh, dAh, dBh, w.rows, 1, w.d, w.n_g, w.m,
-                                 w.n, w.dtype, scratch, need, chunk, stream=s)
+        sums = torch.empty(w.n_g, w.m + 1 + w.n, dtype=torch.float64, device="cuda")
+        st = grk.grkan_step_host(xh, dyh, a, b, yh, dxh, dAh, dBh, sums, w.rows, 1, w.d, w.n_g,
+                                 w.m, w.n, w.dtype, scratch, need, chunk, stream=s)
         assert st == 0, grk.grkan_last_error()
         s.synchronize()
         xd, dyd = xh.cuda(), dyh.cuda()
@@ -45,6 +46,17 @@ def test_host_step_matches_device_calls(name, rows, chunk):
         torch.cuda.synchronize()
         assert torch.equal(yh, y.cpu()) and torch.equal(dxh, dx.cpu())
         assert torch.equal(dAh, dA.cpu()) and torch.equal(dBh, dB.cpu())
+        # the float64 sums are the ones grkan_backward_merge gives for the batch
+        wsb = grk.grkan_backward_workspace_bytes(w.rows, 1, w.d, w.n_g, w.m, w.n, w.dtype)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        dx2 = torch.empty_like(xd)
+        ref = torch.empty_like(sums)
+        assert grk.grkan_backward_partials(xd, dyd, a, b, dx2, w.rows, 1, w.d, w.n_g, w.m, w.n,
+                                           w.dtype, ws, wsb, 0) == 0
+        assert grk.grkan_backward_merge(ws, wsb, dA, dB, ref, w.rows, 1, w.d, w.n_g, w.m, w.n,
+                                        w.dtype) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(sums, ref)
 
 
 def test_host_step_rejects_small_scratch():
@@ -55,6 +67,6 @@ def test_host_step_rejects_small_scratch():
     scratch = torch.empty(need, dtype=torch.uint8, device="cuda")
     dA = torch.empty(8, 6).pin_memory()
     dB = torch.empty(8, 4).pin_memory()
-    st = grk.grkan_step_host(x, x, a, b, x, x, dA, dB, 4, 1, 64, 8, 5, 4, grk.F32, scratch,
+    st = grk.grkan_step_host(x, x, a, b, x, x, dA, dB, None, 4, 1, 64, 8, 5, 4, grk.F32, scratch,
                              need - 256, 0)
     assert st == 5
