@@ -51,9 +51,14 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused-launches", type=int, default=50,
                     help="launches of the recompute variant timed after the step (0: skip)")
-    ap.add_argument("--linear-nout", type=int, default=0,
+    ap.add_argument("--linear-nout", type=int, default=768,
                     help="also time the activation fused into a following linear layer with "
-                         "this many outputs (bf16 workloads; 0: skip)")
+                         "this many outputs (bf16 workloads; default 768, the KAT-B MLP's "
+                         "second linear layer; 0: skip)")
+    ap.add_argument("--per-config", default="kat_t,kat_s,stress:1,stress:8,stress:64",
+                    help="other workloads timed after the main step (name[:n_g], comma "
+                         "separated; empty: skip)")
+    ap.add_argument("--per-config-steps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -203,6 +208,90 @@ def run_reference(args, w):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
+
+
+# --- other workloads, timed after the main step ----------------------------------------
+
+def time_workload(grk, torch, dev, w, steps, peak):
+    """Forward, backward and step times of one workload on device-resident inputs
+    (CUDA events per kernel, medians over `steps` steps after 3 warm-ups), plus
+    the one-pass forward + backward."""
+    B, N, d, n_g, m, n, dt = w.B, w.N, w.d, w.n_g, w.m, w.n, w.dtype
+    E = w.elems
+    tdt = torch.float32 if dt == synth.F32 else torch.bfloat16
+    xh = torch.empty((B, N, d), dtype=tdt, pin_memory=True)
+    gh = torch.empty((B, N, d), dtype=tdt, pin_memory=True)
+    synth.fill_ptr(xh.data_ptr(), E, dt, w.seed, synth.X_STREAM, w.x_kind, w.x_scale, w.x_clip)
+    synth.fill_ptr(gh.data_ptr(), E, dt, w.seed, synth.DY_STREAM, synth.KIND_NORMAL, w.dy_scale)
+    x, dy = xh.to(dev), gh.to(dev)
+    del xh, gh
+    a_np, b_np = w.coefficients()
+    a, b = torch.from_numpy(a_np).to(dev), torch.from_numpy(b_np).to(dev)
+    y, dx = torch.empty_like(x), torch.empty_like(x)
+    dA = torch.empty((n_g, m + 1), dtype=torch.float32, device=dev)
+    dB = torch.empty((n_g, n), dtype=torch.float32, device=dev)
+    wsb = grk.grkan_backward_workspace_bytes(B, N, d, n_g, m, n, dt)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def ok(st, what):
+        if st != 0:
+            raise grk.GrkanError(st, what)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ok(grk.grkan_forward(x, y, a, b, B, N, d, n_g, m, n, dt, sp), "forward")
+        if ev is not None:
+            ev[1].record(stream)
+        ok(grk.grkan_backward_partials(x, dy, a, b, dx, B, N, d, n_g, m, n, dt, ws, wsb, 0, sp),
+           "backward_partials")
+        if ev is not None:
+            ev[2].record(stream)
+        ok(grk.grkan_backward_merge(ws, wsb, dA, dB, None, B, N, d, n_g, m, n, dt, sp), "merge")
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(3):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for k in range(steps):
+        step(evs[k])
+    torch.cuda.synchronize(dev)
+    fwd = float(np.median([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd = float(np.median([e[1].elapsed_time(e[2]) for e in evs]))
+    stp = float(np.median([e[0].elapsed_time(e[3]) for e in evs]))
+
+    def one_pass():
+        ok(grk.grkan_forward_backward(x, dy, a, b, y, dx, dA, dB, B, N, d, n_g, m, n, dt, ws, wsb,
+                                      0, sp), "forward_backward")
+    for _ in range(3):
+        one_pass()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(steps):
+        one_pass()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    fb = f0.elapsed_time(f1) / steps
+
+    def rates(kind, ms):
+        by = accounting.bytes_per_element(kind, dt) * E
+        return {"ms": ms, "GB/s": by / (ms * 1e-3) / 1e9, "frac": by / (ms * 1e-3) / 1e9 / peak,
+                "frac_of_8TBps": by / (ms * 1e-3) / 8e12}
+    out = {"workload": w.name, "dtype": dtype_name(w), "shape": [B, N, d], "n_g": n_g,
+           "elements": E, "elements_per_s": E / (stp * 1e-3),
+           "forward": rates("forward", fwd), "backward_stage1": rates("backward", bwd),
+           "step": rates("step", stp), "forward_backward_recompute": rates("forward_backward", fb),
+           "kernel_path": {"forward": "tma" if grk.grkan_forward_path(
+               x, y, B, N, d, n_g, m, n, dt) == 1 else "generic",
+               "backward": "tma" if grk.grkan_backward_path(
+               x, dy, dx, B, N, d, n_g, m, n, dt) == 1 else "generic"}}
+    del x, dy, y, dx, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 # --- our arm ---------------------------------------------------------------------------
@@ -402,6 +491,18 @@ def main():
                     "torch.matmul (cuBLAS) + grkan_backward; weight gradient not included"}
         del Wl, outl, dout, dyl, wsl
 
+    # the other workloads (KAT-T, KAT-S, the group stress sweep), each timed on its
+    # own device-resident inputs after the main step; not part of `value`
+    per_config = None
+    if args.per_config and world == 1:
+        peak_gbs = peaks()[0]
+        per_config = []
+        for item in [c for c in args.per_config.split(",") if c]:
+            cname, _, cng = item.partition(":")
+            cw = synth.workload(cname, n_g=int(cng) if cng else None)
+            per_config.append(time_workload(grk, torch, dev, cw, args.per_config_steps,
+                                            peak_gbs))
+
     # end to end through the C ABI's host-buffer entry point: pinned inputs in,
     # y, dx and dA/dB out, copies inside the timed region (chunks streamed over
     # three streams so that copies in, kernels and copies out overlap)
@@ -469,8 +570,12 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "backward stage 1 (dx + dA/dB partials)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": measured_traffic(w),
-                     "traffic_note": "ncu dram read+write of a 25,000-row capture scaled by "
-                                     "elements (profiles/bwd_tma_kat_b.md)",
+                     "traffic_note": "ncu dram__bytes_read + dram__bytes_write of one launch "
+                                     "on the first 25,000 rows, scaled by elements "
+                                     "(profiles/bwd_tma_kat_b.md): reads equal the "
+                                     "algorithmic x + dy bytes; writes come out below the "
+                                     "algorithmic dx bytes because the capture's last dx "
+                                     "lines are still in L2 when the kernel ends",
                      "peak_source": peak_src,
                      "bytes_per_launch": bwd_bytes, "launch_ms": bwd_ms},
         # the backward kernel is bound by FP32 arithmetic, not HBM: the same
@@ -494,8 +599,10 @@ def main():
             "forward_backward_recompute": None if fused_ms is None else {
                 "ms": fused_ms, "GB/s": fused_bytes / (fused_ms * 1e-3) / 1e9,
                 "frac": fused_bytes / (fused_ms * 1e-3) / 1e9 / peak,
-                "note": "y, dx and dA/dB from one pass over x and dy, merge included; "
-                        "not part of the timed step"},
+                "frac_of_8TBps": fused_bytes / (fused_ms * 1e-3) / 8e12,
+                "note": "y, dx and dA/dB from one pass over x and dy (4 element sizes per "
+                        "element), merge included; activation-recompute training only, not "
+                        "part of the timed step"},
             "step": {"ms": ms_step, "GB/s": step_bytes / (ms_step * 1e-3) / 1e9,
                      "frac": step_bytes / (ms_step * 1e-3) / 1e9 / peak,
                      "frac_of_8TBps": step_bytes / (ms_step * 1e-3) / 8e12},
@@ -505,6 +612,7 @@ def main():
                 "d2h_bytes_per_step": 2 * nbytes + (n_g * K) * 4, "ms_per_step": e2e_ms,
                 "api": "grkan_step_host (x, dy in; y, dx, dA, dB out; pinned host buffers)"},
         "fused_linear": linear,
+        "per_config": per_config,
         "gpu_launches": args.steps * (3 + (1 if world > 1 else 0)),
         "clocks": clocks,
         "device_error": derr,

@@ -296,12 +296,14 @@ grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float
 grkan_status_t launch_tma_bwd(const Plan& p, const void* x, const void* dy, void* dx, void* y,
                               const float* a, const float* b, float* ws, long long ws_T,
                               long long tile0, cudaStream_t st) {
-  CUtensorMap mx, mdy;
-  if (!make_map(&mx, x, p, p.bbox) || !make_map(&mdy, dy, p, p.bbox)) return GRKAN_ERR_CUDA;
+  CUtensorMap mx, mdy, mdx;
+  if (!make_map(&mx, x, p, p.bbox) || !make_map(&mdy, dy, p, p.bbox) ||
+      !make_map(&mdx, dx, p, p.bbox))
+    return GRKAN_ERR_CUDA;
   grk::TmaGeom geom = make_geom(p, p.bbox);
   geom.ws_T = ws_T;
   geom.ws_tile0 = tile0;
-  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, dx, y, a, b, ws,
+  cudaError_t e = grk::launch_bwd_tma(p.dtype == GRKAN_BF16, geom, mx, mdy, mdx, dx, y, a, b, ws,
                                       sm_count(), st);
   return cuda_status(e, "backward (TMA) launch");
 }

@@ -14,7 +14,8 @@
 //     mixed-radix cursors;
 //   - the lanes evaluate the rational function on pairs of elements with packed
 //     float32x2 arithmetic from coefficients kept in a CTA-wide table, and write
-//     y or dx with 16-byte streaming stores;
+//     y or dx with 16-byte streaming stores (the float32 backward stages dx in a
+//     per-warp slot and writes it with one TMA tensor store per box);
 //   - the backward keeps the m + 1 + n coefficient-gradient sums in registers;
 //     at the end of a unit the warp folds them in a fixed order (recursive
 //     halving over shuffles) into one float32 partial per (unit, coefficient)
@@ -103,6 +104,18 @@ struct TmaGeom {
 #define GRK_BF16_BWD_STAGES 2
 #endif
 
+// How the backward writes dx, per element type: 0 = 16-byte streaming stores
+// from the lanes (each pass's values first, then its stores, each guarded by its
+// row); 2 = the lanes stage the box in a shared-memory slot and one TMA tensor
+// store per box writes it (rows past the tensor are clipped by the tensor map).
+// Measured on B200: bf16 (arithmetic-bound) is fastest with 0, float32
+// (HBM-bound) with 2.
+#ifndef GRK_F32_BWD_STORE
+#define GRK_F32_BWD_STORE 2
+#endif
+#ifndef GRK_BF16_BWD_STORE
+#define GRK_BF16_BWD_STORE 0
+#endif
 constexpr int kFwdWarps = GRK_FWD_WARPS;  // forward: 16 warps x 128 registers
 constexpr int kFwdThreads = kFwdWarps * 32;
 
@@ -116,6 +129,7 @@ struct Shape<IoF32> {
   static constexpr int kBwdHalves = GRK_F32_BWD_HALVES;  // passes over a backward box
   static constexpr int kBwdStages = GRK_F32_BWD_STAGES;  // backward ring depth
   static constexpr int kBwdWarps = GRK_F32_BWD_WARPS;    // backward warps per CTA
+  static constexpr int kBwdStore = GRK_F32_BWD_STORE;    // how dx is written (see above)
 };
 template <>
 struct Shape<IoBF16> {
@@ -125,6 +139,7 @@ struct Shape<IoBF16> {
   static constexpr int kBwdHalves = GRK_BF16_BWD_HALVES;
   static constexpr int kBwdStages = GRK_BF16_BWD_STAGES;
   static constexpr int kBwdWarps = GRK_BF16_BWD_WARPS;
+  static constexpr int kBwdStore = GRK_BF16_BWD_STORE;
 };
 template <class IO>
 constexpr unsigned fwd_box_bytes() {
@@ -231,6 +246,27 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+
+// TMA tensor store of a box from shared memory (bulk async-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1,
+                                             uint32_t src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk store has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk store is complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -531,12 +567,14 @@ __device__ __forceinline__ void load_coef(bool use_tab, const float* tab, const 
 struct WarpLayout {
   unsigned box_slot;   // bytes of one box slot
   unsigned stage;      // bytes of one stage (all tensors)
+  unsigned out_off;    // output staging slots (boxes written back by TMA stores)
   unsigned bar_off;    // full[stages] then empty[stages]
   unsigned per_warp;   // bytes per warp (multiple of 128)
-  __host__ __device__ WarpLayout(unsigned box_bytes, int tensors, int stages) {
+  __host__ __device__ WarpLayout(unsigned box_bytes, int tensors, int stages, int outs = 0) {
     box_slot = round_up(box_bytes, 128);
     stage = box_slot * (unsigned)tensors;
-    bar_off = stage * (unsigned)stages;
+    out_off = stage * (unsigned)stages;
+    bar_off = out_off + box_slot * (unsigned)outs;
     per_warp = round_up(bar_off + (unsigned)(2 * stages) * 8, 128);
   }
 };
@@ -774,6 +812,7 @@ __device__ __forceinline__ int tile_row_blocks(const TmaGeom& g, long long tile)
 template <class IO, int M, int N, bool kWithY, bool kFull>
 __global__ void __launch_bounds__(Shape<IO>::kBwdWarps * 32, 1)
 bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdy,
+        const __grid_constant__ CUtensorMap mdx,
         typename IO::T* __restrict__ dx, typename IO::T* __restrict__ yout,
         const float* __restrict__ a,
         const float* __restrict__ b, float* __restrict__ ws, const TmaGeom geom) {
@@ -787,7 +826,8 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const WarpLayout L(geom.box_bytes, 2, S_::kBwdStages);
+  constexpr bool kTmaOut = S_::kBwdStore == 2;  // dx leaves through a staging slot and TMA
+  const WarpLayout L(geom.box_bytes, 2, S_::kBwdStages, kTmaOut ? 1 : 0);
   unsigned char* base = smem + warp * L.per_warp;
   float* ctab = reinterpret_cast<float*>(smem + S_::kBwdWarps * L.per_warp);
   const bool use_tab = geom.n_g <= kTableGroups;
@@ -809,6 +849,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     if (warp == 0) {
       prefetch_map(&mx);
       prefetch_map(&mdy);
+      if (kTmaOut) prefetch_map(&mdx);
     }
   }
   if (use_tab) build_coef_table<M, N>(ctab, a, b, geom.n_g);
@@ -905,6 +946,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
         const long long box_off = (long long)r0 * row_bytes + (long long)bx * geom.bw * sizeof(T);
         char* dxo = dxt + box_off;
         char* yo = kWithY ? yt + box_off : nullptr;
+        uint4* outs = reinterpret_cast<uint4*>(base + L.out_off) + lane;  // staging (kTmaOut)
 #pragma unroll
         for (int h = 0; h < kPasses; ++h) {
           uint4 xv[kBwdVec], gv[kBwdVec];
@@ -934,6 +976,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
               }
             }
           }
+          uint4 ov[kBwdVec], oyv[kBwdVec];
 #pragma unroll
           for (int it = 0; it < kBwdVec; ++it) {
             const int sl = h * kBwdVec + it;
@@ -968,10 +1011,42 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
                 oy = make_uint4(__float_as_uint(y0.x), __float_as_uint(y0.y),
                                 __float_as_uint(y1.x), __float_as_uint(y1.y));
             }
-            if (lm.row[sl] < lim) {
-              store16(dxo + boff[sl], o);
-              if constexpr (kWithY) store16(yo + boff[sl], oy);
+            ov[it] = o;
+            if constexpr (kWithY) oyv[it] = oy;
+          }
+          if constexpr (kTmaOut) {
+            // the slot is free once the previous box's store has read it
+            if (h == 0) {
+              if (lane == 0) bulk_wait_read_all();
+              __syncwarp();
             }
+#pragma unroll
+            for (int it = 0; it < kBwdVec; ++it) {
+              const int sl = h * kBwdVec + it;
+              if (kFull || lm.row[sl] < geom.SCw) outs[32 * sl] = ov[it];
+              if constexpr (kWithY)
+                if (lm.row[sl] < lim) store16(yo + boff[sl], oyv[it]);
+            }
+          } else {
+#pragma unroll
+            for (int it = 0; it < kBwdVec; ++it) {
+              const int sl = h * kBwdVec + it;
+              if (lm.row[sl] < lim) {
+                store16(dxo + boff[sl], ov[it]);
+                if constexpr (kWithY) store16(yo + boff[sl], oyv[it]);
+              }
+            }
+          }
+        }
+        if constexpr (kTmaOut) {
+          // the lanes' shared-memory writes become visible to the async proxy,
+          // then one store writes the box (rows past the tensor are clipped)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&mdx, g * geom.dg + bx * geom.bw, (int)(tile * geom.S) + r0,
+                         smem_addr(base + L.out_off));
+            bulk_commit();
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -994,6 +1069,7 @@ bwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
       if (!mbar_wait(full0 + 8 * (j % S_::kBwdStages), (uint32_t)(j / S_::kBwdStages) & 1))
         report(kErrDrainWait);
   }
+  if (kTmaOut && lane == 0) bulk_wait_all();  // stores done before the CTA's memory goes
 }
 
 // --- host-side launchers ---------------------------------------------------------
@@ -1027,7 +1103,10 @@ inline unsigned fwd_smem_bytes() {
 }
 template <class IO, int M, int N>
 inline unsigned bwd_smem_bytes() {
-  return Shape<IO>::kBwdWarps * WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages).per_warp +
+  return Shape<IO>::kBwdWarps *
+             WarpLayout(bwd_box_bytes<IO>(), 2, Shape<IO>::kBwdStages,
+                        Shape<IO>::kBwdStore == 2 ? 1 : 0)
+                 .per_warp +
          coef_table_bytes<M, N>();
 }
 
@@ -1059,48 +1138,55 @@ inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap
 
 template <class IO, int M, int N, bool kWithY, bool kFull>
 inline cudaError_t launch_bwd_tma_t(const TmaGeom& g, const CUtensorMap& mx,
-                                    const CUtensorMap& mdy, void* dx, void* y, const float* a,
-                                    const float* b, float* ws, long long grid, cudaStream_t st) {
+                                    const CUtensorMap& mdy, const CUtensorMap& mdx, void* dx,
+                                    void* y, const float* a, const float* b, float* ws,
+                                    long long grid, cudaStream_t st) {
   const unsigned smem = bwd_smem_bytes<IO, M, N>();
   cudaError_t e = ensure_smem<bwd_tma<IO, M, N, kWithY, kFull>>(smem);
   if (e != cudaSuccess) return e;
   bwd_tma<IO, M, N, kWithY, kFull><<<(unsigned)grid, Shape<IO>::kBwdWarps * 32, smem, st>>>(
-      mx, mdy, (typename IO::T*)dx, (typename IO::T*)y, a, b, ws, g);
+      mx, mdy, mdx, (typename IO::T*)dx, (typename IO::T*)y, a, b, ws, g);
   return cudaGetLastError();
 }
 
 template <class IO, int M, int N>
 inline cudaError_t launch_bwd_tma_io(const TmaGeom& g, const CUtensorMap& mx,
-                                     const CUtensorMap& mdy, void* dx, void* y, const float* a,
-                                     const float* b, float* ws, long long grid, cudaStream_t st) {
+                                     const CUtensorMap& mdy, const CUtensorMap& mdx, void* dx,
+                                     void* y, const float* a, const float* b, float* ws,
+                                     long long grid, cudaStream_t st) {
   // every lane vector slot used: the box is exactly 32 lanes x NV vectors
   const bool full = g.box_bytes == bwd_box_bytes<IO>();
   if (y) {
     if constexpr (M == 5 && N == 4) {
-      return full ? launch_bwd_tma_t<IO, M, N, true, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-                  : launch_bwd_tma_t<IO, M, N, true, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+      return full ? launch_bwd_tma_t<IO, M, N, true, true>(g, mx, mdy, mdx, dx, y, a, b, ws, grid,
+                                                            st)
+                  : launch_bwd_tma_t<IO, M, N, true, false>(g, mx, mdy, mdx, dx, y, a, b, ws,
+                                                             grid, st);
     } else {
       return cudaErrorNotSupported;
     }
   }
-  return full ? launch_bwd_tma_t<IO, M, N, false, true>(g, mx, mdy, dx, y, a, b, ws, grid, st)
-              : launch_bwd_tma_t<IO, M, N, false, false>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+  return full ? launch_bwd_tma_t<IO, M, N, false, true>(g, mx, mdy, mdx, dx, y, a, b, ws, grid, st)
+              : launch_bwd_tma_t<IO, M, N, false, false>(g, mx, mdy, mdx, dx, y, a, b, ws, grid,
+                                                          st);
 }
 
 // y == nullptr: backward only; otherwise also write the recomputed forward y
-// (degree (5, 4) only).
+// (degree (5, 4) only). mdx maps dx with the backward box (used when dx is
+// written by TMA stores).
 inline cudaError_t launch_bwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
-                                  const CUtensorMap& mdy, void* dx, void* y, const float* a,
-                                  const float* b, float* ws, int sms, cudaStream_t st) {
+                                  const CUtensorMap& mdy, const CUtensorMap& mdx, void* dx,
+                                  void* y, const float* a, const float* b, float* ws, int sms,
+                                  cudaStream_t st) {
   if (g.box_bytes > bwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long units = g.T * g.n_g;
   const int warps = bf16 ? Shape<IoBF16>::kBwdWarps : Shape<IoF32>::kBwdWarps;
   long long grid = sms;
   if (grid * warps > units) grid = (units + warps - 1) / warps;
-#define GRK_BWD_CASE(M, N)                                                              \
-  if (g.m == M && g.n == N)                                                             \
-    return bf16 ? launch_bwd_tma_io<IoBF16, M, N>(g, mx, mdy, dx, y, a, b, ws, grid, st) \
-                : launch_bwd_tma_io<IoF32, M, N>(g, mx, mdy, dx, y, a, b, ws, grid, st);
+#define GRK_BWD_CASE(M, N)                                                                   \
+  if (g.m == M && g.n == N)                                                                  \
+    return bf16 ? launch_bwd_tma_io<IoBF16, M, N>(g, mx, mdy, mdx, dx, y, a, b, ws, grid, st) \
+                : launch_bwd_tma_io<IoF32, M, N>(g, mx, mdy, mdx, dx, y, a, b, ws, grid, st);
   GRK_TMA_DEGREES(GRK_BWD_CASE)
 #undef GRK_BWD_CASE
   return cudaErrorNotSupported;
