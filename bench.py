@@ -99,16 +99,58 @@ def dtype_name(w):
 # --- clocks ---------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and throttle reasons sampled during the timed region: through NVML
+    every 2 ms in a background thread when the bindings are there (a timed region
+    of a few milliseconds still gets several samples), else `nvidia-smi -lms 100`.
+    Read-only: nothing here changes a setting of the GPU."""
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_id):
+    def __init__(self, gpu_id, interval_s=0.002):
         self.gpu_id = gpu_id
+        self.interval = interval_s
         self.proc = None
+        self.thread = None
         self.path = os.path.join(tempfile.gettempdir(), "grkan_clocks_%d.csv" % os.getpid())
 
+    def _nvml_loop(self, nv, h, bits):
+        import threading
+        sm, mx, reasons = [], [], set()
+        maxc = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_flag.is_set():
+            try:
+                sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                mx.append(float(maxc))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, bit in bits.items():
+                    if r & bit:
+                        reasons.add(name)
+            except Exception:
+                pass
+            self.stop_flag.wait(self.interval)
+        self.result = (sm, mx, reasons)
+
     def start(self):
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            bits = {"hw_slowdown": nv.nvmlClocksThrottleReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksThrottleReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksThrottleReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksThrottleReasonSwPowerCap}
+            self.stop_flag = threading.Event()
+            self.result = None
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, bits),
+                                           daemon=True)
+            self.thread.start()
+            self.source = "nvml, every %.0f ms" % (self.interval * 1e3)
+            return
+        except Exception:
+            self.thread = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
@@ -116,11 +158,22 @@ class ClockSampler:
                 ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
                  "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, every 100 ms"
             time.sleep(0.3)
         except Exception:
             self.proc = None
 
+    def _summary(self, sm, mx, reasons):
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "samples": len(sm), "reasons": sorted(reasons), "source": self.source}
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            return self._summary(*self.result) if self.result else None
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -130,7 +183,6 @@ class ClockSampler:
             self.proc.kill()
         self.f.close()
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
@@ -140,13 +192,10 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[4:8]):
+            for nm, v in zip(self.REASONS, parts[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return self._summary(sm, mx, reasons)
 
 
 # --- reference arm / CPU baseline: the fp64 oracle on host cores ----------------------

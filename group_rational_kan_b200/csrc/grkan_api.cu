@@ -286,10 +286,11 @@ int sm_count() {
 
 grkan_status_t launch_tma_fwd(const Plan& p, const void* x, void* y, const float* a,
                               const float* b, cudaStream_t st) {
-  CUtensorMap mx;
-  if (!make_map(&mx, x, p, p.fbox)) return GRKAN_ERR_CUDA;
+  CUtensorMap mx, my;
+  if (!make_map(&mx, x, p, p.fbox) || !make_map(&my, y, p, p.fbox)) return GRKAN_ERR_CUDA;
   const grk::TmaGeom geom = make_geom(p, p.fbox);
-  cudaError_t e = grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, y, a, b, sm_count(), st);
+  cudaError_t e =
+      grk::launch_fwd_tma(p.dtype == GRKAN_BF16, geom, mx, my, y, a, b, sm_count(), st);
   return cuda_status(e, "forward (TMA) launch");
 }
 

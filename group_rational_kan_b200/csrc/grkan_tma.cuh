@@ -59,11 +59,12 @@ struct TmaGeom {
 // float32, HBM-bound, and 12 in bf16, whose arithmetic-bound loop runs faster with
 // up to 168 registers per thread). Every warp owns, per element
 // type, a ring of forward stages (one box of x each) and of backward stages
-// (one box of x and one of dy each). float32 rows are HBM-bound: smaller boxes,
-// deeper rings. The bf16 forward streams 1.5 KiB boxes through four stages
-// (measured faster than 2 KiB x 6). The bf16 backward is bound by arithmetic
-// issue: 3 KiB boxes read in three passes of two 16-byte vectors per lane, two
-// stages.
+// (one box of x and one of dy each). The float32 forward streams 3 KiB boxes
+// through three stages beside a staging slot for its TMA stores; the float32
+// backward, 1.5 KiB boxes through four. The bf16 forward streams 1.5 KiB boxes
+// through four stages (measured faster than 2 KiB x 6). The bf16 backward is
+// bound by arithmetic issue: 3 KiB boxes read in three passes of two 16-byte
+// vectors per lane, two stages.
 #ifndef GRK_FWD_WARPS
 #define GRK_FWD_WARPS 16
 #endif
@@ -77,7 +78,7 @@ struct TmaGeom {
 #define GRK_F32_FWD_VEC 6
 #endif
 #ifndef GRK_F32_FWD_STAGES
-#define GRK_F32_FWD_STAGES 4
+#define GRK_F32_FWD_STAGES 3
 #endif
 #ifndef GRK_F32_BWD_VEC
 #define GRK_F32_BWD_VEC 3
@@ -116,6 +117,17 @@ struct TmaGeom {
 #ifndef GRK_BF16_BWD_STORE
 #define GRK_BF16_BWD_STORE 0
 #endif
+// How the forward writes y: 0 = each vector computed and stored under its row
+// guard; 1 = all of a box's values first, then the guarded stores (bf16: 2.5 %
+// faster than 0 on B200); 2 = staged and written by one TMA store per box
+// (float32, with three ring stages to make room for the slot: 3-4 % faster than
+// 0 with four).
+#ifndef GRK_F32_FWD_STORE
+#define GRK_F32_FWD_STORE 2
+#endif
+#ifndef GRK_BF16_FWD_STORE
+#define GRK_BF16_FWD_STORE 1
+#endif
 constexpr int kFwdWarps = GRK_FWD_WARPS;  // forward: 16 warps x 128 registers
 constexpr int kFwdThreads = kFwdWarps * 32;
 
@@ -130,6 +142,7 @@ struct Shape<IoF32> {
   static constexpr int kBwdStages = GRK_F32_BWD_STAGES;  // backward ring depth
   static constexpr int kBwdWarps = GRK_F32_BWD_WARPS;    // backward warps per CTA
   static constexpr int kBwdStore = GRK_F32_BWD_STORE;    // how dx is written (see above)
+  static constexpr int kFwdStore = GRK_F32_FWD_STORE;    // how y is written (see above)
 };
 template <>
 struct Shape<IoBF16> {
@@ -140,6 +153,7 @@ struct Shape<IoBF16> {
   static constexpr int kBwdStages = GRK_BF16_BWD_STAGES;
   static constexpr int kBwdWarps = GRK_BF16_BWD_WARPS;
   static constexpr int kBwdStore = GRK_BF16_BWD_STORE;
+  static constexpr int kFwdStore = GRK_BF16_FWD_STORE;
 };
 template <class IO>
 constexpr unsigned fwd_box_bytes() {
@@ -672,14 +686,15 @@ struct Cursor3 {
 
 template <class IO, int M, int N>
 __global__ void __launch_bounds__(kFwdThreads, 1)
-fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
+fwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap my,
+        typename IO::T* __restrict__ y,
         const float* __restrict__ a, const float* __restrict__ b, const TmaGeom geom) {
   using S_ = Shape<IO>;
   using D = Deg<M, N>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const WarpLayout L(geom.box_bytes, 1, S_::kFwdStages);
+  const WarpLayout L(geom.box_bytes, 1, S_::kFwdStages, S_::kFwdStore == 2 ? 1 : 0);
   unsigned char* base = smem + warp * L.per_warp;
   float* ctab = reinterpret_cast<float*>(smem + kFwdWarps * L.per_warp);
   const bool use_tab = geom.n_g <= kTableGroups;
@@ -699,7 +714,10 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
-    if (warp == 0) prefetch_map(&mx);
+    if (warp == 0) {
+      prefetch_map(&mx);
+      if (S_::kFwdStore == 2) prefetch_map(&my);
+    }
   }
   if (use_tab) build_coef_table<M, N>(ctab, a, b, geom.n_g);
   __syncthreads();
@@ -760,24 +778,50 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
     }
     const long long row0 = cc.hi * geom.SCw;
     typename IO::T* yo = y + row0 * geom.d + (g * geom.dg + cc.lo * geom.bw);
+    auto fwd_vec = [&](const uint4& xv) {
+      uint4 o;
+      if constexpr (IO::kBytes == 2) {
+        o.x = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(xv.x)));
+        o.y = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(xv.y)));
+        o.z = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(xv.z)));
+        o.w = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(xv.w)));
+      } else {
+        const float2 p0 = D::fwd(c, make_float2(__uint_as_float(xv.x), __uint_as_float(xv.y)));
+        const float2 p1 = D::fwd(c, make_float2(__uint_as_float(xv.z), __uint_as_float(xv.w)));
+        o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
+                       __float_as_uint(p1.y));
+      }
+      return o;
+    };
+    if constexpr (S_::kFwdStore == 0) {
 #pragma unroll
-    for (int it = 0; it < S_::kFwdVec; ++it) {
-      if (row0 + lm.row[it] < geom.rows) {
-        uint4 o;
-        if constexpr (IO::kBytes == 2) {
-          o.x = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].x)));
-          o.y = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].y)));
-          o.z = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].z)));
-          o.w = f2_to_bf16x2(D::fwd(c, bf16x2_to_f2(v[it].w)));
-        } else {
-          const float2 p0 =
-              D::fwd(c, make_float2(__uint_as_float(v[it].x), __uint_as_float(v[it].y)));
-          const float2 p1 =
-              D::fwd(c, make_float2(__uint_as_float(v[it].z), __uint_as_float(v[it].w)));
-          o = make_uint4(__float_as_uint(p0.x), __float_as_uint(p0.y), __float_as_uint(p1.x),
-                         __float_as_uint(p1.y));
-        }
-        store16(yo + lm.off[it], o);
+      for (int it = 0; it < S_::kFwdVec; ++it)
+        if (row0 + lm.row[it] < geom.rows) store16(yo + lm.off[it], fwd_vec(v[it]));
+    } else if constexpr (S_::kFwdStore == 1) {
+      // every vector's values first (rows past the tensor arrive zero-filled),
+      // then the guarded stores: the arithmetic stays one basic block
+      uint4 o[S_::kFwdVec];
+#pragma unroll
+      for (int it = 0; it < S_::kFwdVec; ++it) o[it] = fwd_vec(v[it]);
+#pragma unroll
+      for (int it = 0; it < S_::kFwdVec; ++it)
+        if (row0 + lm.row[it] < geom.rows) store16(yo + lm.off[it], o[it]);
+    } else {
+      // staged in the warp's output slot, written by one TMA store (clipped rows)
+      uint4 o[S_::kFwdVec];
+#pragma unroll
+      for (int it = 0; it < S_::kFwdVec; ++it) o[it] = fwd_vec(v[it]);
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      uint4* outs = reinterpret_cast<uint4*>(base + L.out_off) + lane;
+#pragma unroll
+      for (int it = 0; it < S_::kFwdVec; ++it)
+        if (lm.row[it] < geom.SCw) outs[32 * it] = o[it];
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&my, g * geom.dg + cc.lo * geom.bw, (int)row0, smem_addr(base + L.out_off));
+        bulk_commit();
       }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -789,6 +833,7 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, typename IO::T* __restrict__ y,
       if (!mbar_wait(full0 + 8 * (j % S_::kFwdStages), (uint32_t)(j / S_::kFwdStages) & 1))
         report(kErrDrainWait);
   }
+  if (S_::kFwdStore == 2 && lane == 0) bulk_wait_all();  // stores done before the CTA ends
 }
 
 // --- backward ------------------------------------------------------------------------
@@ -1098,7 +1143,10 @@ inline cudaError_t ensure_smem(unsigned bytes) {
 // the coefficient table.
 template <class IO, int M, int N>
 inline unsigned fwd_smem_bytes() {
-  return kFwdWarps * WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages).per_warp +
+  return kFwdWarps *
+             WarpLayout(fwd_box_bytes<IO>(), 1, Shape<IO>::kFwdStages,
+                        Shape<IO>::kFwdStore == 2 ? 1 : 0)
+                 .per_warp +
          coef_table_bytes<M, N>();
 }
 template <class IO, int M, int N>
@@ -1111,26 +1159,29 @@ inline unsigned bwd_smem_bytes() {
 }
 
 template <class IO, int M, int N>
-inline cudaError_t launch_fwd_tma_t(const TmaGeom& g, const CUtensorMap& mx, void* y,
-                                    const float* a, const float* b, long long grid,
-                                    cudaStream_t st) {
+inline cudaError_t launch_fwd_tma_t(const TmaGeom& g, const CUtensorMap& mx,
+                                    const CUtensorMap& my, void* y, const float* a,
+                                    const float* b, long long grid, cudaStream_t st) {
   const unsigned smem = fwd_smem_bytes<IO, M, N>();
   cudaError_t e = ensure_smem<fwd_tma<IO, M, N>>(smem);
   if (e != cudaSuccess) return e;
-  fwd_tma<IO, M, N><<<(unsigned)grid, kFwdThreads, smem, st>>>(mx, (typename IO::T*)y, a, b, g);
+  fwd_tma<IO, M, N><<<(unsigned)grid, kFwdThreads, smem, st>>>(mx, my, (typename IO::T*)y, a, b,
+                                                                g);
   return cudaGetLastError();
 }
 
-inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx, void* y,
-                                  const float* a, const float* b, int sms, cudaStream_t st) {
+// my maps y with the forward box (used when y is written by TMA stores).
+inline cudaError_t launch_fwd_tma(bool bf16, const TmaGeom& g, const CUtensorMap& mx,
+                                  const CUtensorMap& my, void* y, const float* a,
+                                  const float* b, int sms, cudaStream_t st) {
   if (g.box_bytes > fwd_box_target(bf16)) return cudaErrorInvalidValue;
   const long long items = ((g.rows + g.SCw - 1) / g.SCw) * g.n_g * g.nbox;
   long long grid = sms;
   if (grid * kFwdWarps > items) grid = (items + kFwdWarps - 1) / kFwdWarps;
 #define GRK_FWD_CASE(M, N)                                                          \
   if (g.m == M && g.n == N)                                                         \
-    return bf16 ? launch_fwd_tma_t<IoBF16, M, N>(g, mx, y, a, b, grid, st)          \
-                : launch_fwd_tma_t<IoF32, M, N>(g, mx, y, a, b, grid, st);
+    return bf16 ? launch_fwd_tma_t<IoBF16, M, N>(g, mx, my, y, a, b, grid, st)      \
+                : launch_fwd_tma_t<IoF32, M, N>(g, mx, my, y, a, b, grid, st);
   GRK_TMA_DEGREES(GRK_FWD_CASE)
 #undef GRK_FWD_CASE
   return cudaErrorNotSupported;
