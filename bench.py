@@ -441,6 +441,10 @@ def main():
     for k in range(args.steps):
         step(evs[k])
     t_end.record(stream)
+    # wait for the end event while letting the clock sampler's thread run (a
+    # blocking synchronize can hold the interpreter for the whole timed region)
+    while not t_end.query():
+        time.sleep(0.0005)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
