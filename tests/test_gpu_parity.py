@@ -32,6 +32,11 @@ CASES = {
     "one_row_bf16": synth.workload("kat_b").with_rows(1),
     "odd_f32_dg10": _custom("odd_f32", 77, 30, 3, 5, 4, synth.F32),
     "odd_bf16_dg6": _custom("odd_bf16", 91, 24, 4, 5, 4, synth.BF16),
+    # TMA-pipelined boxes that do not fill every lane's vector slots (40-channel
+    # groups: 9-row float32 / 38-row bf16 backward boxes), through the staged
+    # TMA stores (float32) and the buffered guarded stores (bf16)
+    "box_partial_f32_dg40": _custom("box_f32_dg40", 301, 160, 4, 5, 4, synth.F32),
+    "box_partial_bf16_dg40": _custom("box_bf16_dg40", 301, 160, 4, 5, 4, synth.BF16),
     "deg_3_2": _custom("deg_3_2", 100, 384, 4, 3, 2, synth.BF16),
     "deg_0_0": _custom("deg_0_0", 60, 64, 2, 0, 0, synth.F32),
     "deg_8_8": _custom("deg_8_8", 60, 64, 4, 8, 8, synth.F32, x_kind=synth.KIND_NORMAL,
@@ -89,7 +94,7 @@ def test_fast_path_is_taken_where_expected():
     for name in ("tiny", "kat_t_ragged", "kat_s_ragged", "kat_b_ragged", "stress_ng1",
                  "stress_ng8", "stress_ng64", "one_row_bf16", "deg_8_8", "deg_3_3_bf16",
                  "deg_4_4_f32", "deg_5_5_bf16", "deg_6_6_f32", "deg_7_7_bf16", "deg_8_8_bf16",
-                 "ng96_bf16", "ng128_f32_deg66"):
+                 "ng96_bf16", "ng128_f32_deg66", "box_partial_f32_dg40", "box_partial_bf16_dg40"):
         w = CASES[name]
         t = torch.empty((w.rows, w.d), dtype=torch.float32 if w.dtype == synth.F32
                         else torch.bfloat16, device="cuda")
@@ -103,7 +108,7 @@ def test_fast_path_is_taken_where_expected():
 
 
 @pytest.mark.parametrize("name", ["kat_b_ragged", "stress_ng64", "kat_t_ragged", "odd_f32_dg10",
-                                  "ng96_bf16", "deg_7_7_bf16"])
+                                  "ng96_bf16", "deg_7_7_bf16", "box_partial_f32_dg40"])
 def test_bitwise_determinism(name):
     w, x, dy, a, b = case_data(name)[:5]
     tx, tdy, ta, tb = _dev(w, x, dy, a, b)
@@ -173,7 +178,8 @@ def test_empty_input_zeroes_gradients():
     assert torch.all(dA == 0) and torch.all(dB == 0)
 
 
-@pytest.mark.parametrize("name", ["kat_b_ragged", "kat_t_ragged", "odd_bf16_dg6"])
+@pytest.mark.parametrize("name", ["kat_b_ragged", "kat_t_ragged", "odd_bf16_dg6",
+                                  "box_partial_f32_dg40"])
 def test_in_place(name):
     w, x, dy, a, b, y_ref, ky, dx_ref, ex, g_ref = case_data(name)
     tx, tdy, ta, tb = _dev(w, x, dy, a, b)
@@ -241,7 +247,8 @@ def test_partials_merge_and_sums64():
 
 @pytest.mark.parametrize("flags", [0, grk.FLAG_GENERIC], ids=["auto", "generic"])
 @pytest.mark.parametrize("name", ["tiny", "kat_t_ragged", "kat_b_ragged", "stress_ng64",
-                                  "one_row_bf16", "odd_f32_dg10", "deg_3_2"])
+                                  "one_row_bf16", "odd_f32_dg10", "deg_3_2",
+                                  "box_partial_f32_dg40", "box_partial_bf16_dg40"])
 def test_fused_recompute_parity(name, flags):
     """grkan_forward_backward (y recomputed inside the backward pass): y against
     the oracle, and dx, dA, dB the same bits as the separate backward call."""
