@@ -119,8 +119,12 @@ class ClockSampler:
         import threading
         sm, mx, reasons = [], [], set()
         maxc = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        self.t_first = self.t_last = None
         while not self.stop_flag.is_set():
             try:
+                now = time.perf_counter()
+                self.t_first = now if self.t_first is None else self.t_first
+                self.t_last = now
                 sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
                 mx.append(float(maxc))
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
@@ -166,8 +170,11 @@ class ClockSampler:
     def _summary(self, sm, mx, reasons):
         if not sm:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "samples": len(sm), "reasons": sorted(reasons), "source": self.source}
+        out = {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+               "samples": len(sm), "reasons": sorted(reasons), "source": self.source}
+        if getattr(self, "t_first", None) is not None:
+            out["window_ms"] = (self.t_last - self.t_first) * 1e3
+        return out
 
     def stop(self):
         if self.thread is not None:
