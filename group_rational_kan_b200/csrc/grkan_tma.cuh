@@ -14,8 +14,9 @@
 //     mixed-radix cursors;
 //   - the lanes evaluate the rational function on pairs of elements with packed
 //     float32x2 arithmetic from coefficients kept in a CTA-wide table, and write
-//     y or dx with 16-byte streaming stores (the float32 backward stages dx in a
-//     per-warp slot and writes it with one TMA tensor store per box);
+//     y or dx with 16-byte streaming stores after computing a pass's values (in
+//     float32 the lanes instead stage the box in a per-warp slot that one TMA
+//     tensor store per box writes out);
 //   - the backward keeps the m + 1 + n coefficient-gradient sums in registers;
 //     at the end of a unit the warp folds them in a fixed order (recursive
 //     halving over shuffles) into one float32 partial per (unit, coefficient)
