@@ -62,8 +62,9 @@ struct TmaGeom {
 // type, a ring of forward stages (one box of x each) and of backward stages
 // (one box of x and one of dy each). The float32 forward streams 3 KiB boxes
 // through three stages beside a staging slot for its TMA stores; the float32
-// backward, 1.5 KiB boxes through four. The bf16 forward streams 1.5 KiB boxes
-// through four stages (measured faster than 2 KiB x 6). The bf16 backward is
+// backward, 1.5 KiB boxes through four. The bf16 forward streams 2 KiB boxes
+// through four stages (measured faster than 1.5 KiB x 4 or x 6, 1 KiB x 8 and
+// 3 KiB x 3). The bf16 backward is
 // bound by arithmetic issue: 3 KiB boxes read in three passes of two 16-byte
 // vectors per lane, two stages.
 #ifndef GRK_FWD_WARPS
@@ -91,7 +92,7 @@ struct TmaGeom {
 #define GRK_F32_BWD_STAGES 4
 #endif
 #ifndef GRK_BF16_FWD_VEC
-#define GRK_BF16_FWD_VEC 3
+#define GRK_BF16_FWD_VEC 4
 #endif
 #ifndef GRK_BF16_FWD_STAGES
 #define GRK_BF16_FWD_STAGES 4
