@@ -116,7 +116,6 @@ class ClockSampler:
         self.path = os.path.join(tempfile.gettempdir(), "grkan_clocks_%d.csv" % os.getpid())
 
     def _nvml_loop(self, nv, h, bits):
-        import threading
         sm, mx, reasons = [], [], set()
         maxc = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         self.t_first = self.t_last = None
@@ -133,7 +132,9 @@ class ClockSampler:
                         reasons.add(name)
             except Exception:
                 pass
+            self.ready.set()
             self.stop_flag.wait(self.interval)
+        self.ready.set()
         self.result = (sm, mx, reasons)
 
     def start(self):
@@ -147,10 +148,12 @@ class ClockSampler:
                     "sw_thermal_slowdown": nv.nvmlClocksThrottleReasonSwThermalSlowdown,
                     "sw_power_cap": nv.nvmlClocksThrottleReasonSwPowerCap}
             self.stop_flag = threading.Event()
+            self.ready = threading.Event()
             self.result = None
             self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, bits),
                                            daemon=True)
             self.thread.start()
+            self.ready.wait(2.0)  # sampling before the timed region starts
             self.source = "nvml, every %.0f ms" % (self.interval * 1e3)
             return
         except Exception:
