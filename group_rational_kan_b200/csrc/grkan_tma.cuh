@@ -763,8 +763,8 @@ fwd_tma(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensor
     const uint4* buf = reinterpret_cast<const uint4*>(base + s * L.stage);
     uint4 v[S_::kFwdVec];
 #pragma unroll
-    for (int it = 0; it < S_::kFwdVec; ++it)
-      if (lm.row[it] < geom.SCw) v[it] = buf[lane + 32 * it];
+    for (int it = 0; it < S_::kFwdVec; ++it)  // slots past the box: zeros, never stored
+      v[it] = lm.row[it] < geom.SCw ? buf[lane + 32 * it] : make_uint4(0u, 0u, 0u, 0u);
     // release the slot and refill it with the item S_::kFwdStages ahead
     __syncwarp();
     if (lane == 0) {
