@@ -623,7 +623,9 @@ def main():
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "dtype_note": "arithmetic type of the kernels (float32, float64 merge); the "
+                      "workload's tensors are config.dtype (%s)" % dtype_name(w),
         "data": "synthetic (seeded counter-based generator; KAT activation shapes)",
         "config": dict(w.describe(), global_batch=B * world, seq_len=N,
                        parallelism="dp%d" % world,
