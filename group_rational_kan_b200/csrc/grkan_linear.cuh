@@ -146,22 +146,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
 
 // Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
 // 64-byte swizzling: rows of 64 bytes, 8-row atoms of 512 bytes one after
@@ -357,7 +341,7 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
           if (col0 >= geom.nout) break;
           const int buf = cb & 1;
           if (cb >= 2) {  // the store that used this buffer has read it
-            if (lane == 0) bulk_wait_read0();
+            if (lane == 0) bulk_wait_read_all();
             __syncwarp();
           }
           unsigned char* sb = stg + buf * kEpiBuf;
@@ -388,11 +372,11 @@ linear_fwd(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUten
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&mo, stg_a + (uint32_t)buf * kEpiBuf, col0, (int)m0 + q * 32);
+            tma_store_2d(&mo, col0, (int)m0 + q * 32, stg_a + (uint32_t)buf * kEpiBuf);
             bulk_commit();
           }
         }
-        if (lane == 0) bulk_wait0();
+        if (lane == 0) bulk_wait_all();
         __syncwarp();
       }
     }

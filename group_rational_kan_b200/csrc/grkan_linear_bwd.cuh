@@ -397,7 +397,7 @@ linear_dgrad(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CU
       }
       tc_fence_after();
       if (i >= 1 && lane == 0) {  // the previous tile's dx stores have read its buffer
-        bulk_wait_read0();
+        bulk_wait_read_all();
         mbar_arrive(xe_bar((i - 1) & 1));
       }
       const bool active = 64 * w3 < ncols;
@@ -443,8 +443,8 @@ linear_dgrad(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CU
         if (lane == 0 && (long long)m0 + 32 * q < geom.rows) {
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh)
-            tma_store_2d(&mdx, xtile_addr(ab) + (uint32_t)(2 * w3 + hh) * kXBox + (uint32_t)q * kXSub,
-                         n0 + 64 * w3 + 32 * hh, m0 + 32 * q);
+            tma_store_2d(&mdx, n0 + 64 * w3 + 32 * hh, m0 + 32 * q,
+                         xtile_addr(ab) + (uint32_t)(2 * w3 + hh) * kXBox + (uint32_t)q * kXSub);
           bulk_commit();
         }
         // the block's partial sums, fixed order: the two lanes of each pair, then
@@ -458,7 +458,7 @@ linear_dgrad(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CU
           ws[((long long)g * 10 + k) * geom.ws_T + slot] = sv[0];
       }
     }
-    if (lane == 0) bulk_wait0();  // this warp's stores are complete
+    if (lane == 0) bulk_wait_all();  // this warp's stores are complete
     __syncwarp();
   }
   // teardown: both CTAs are done with the accumulators and with each other's
