@@ -16,11 +16,17 @@ import torch.distributed as dist
 
 
 def all_gather_sums(sums64: torch.Tensor, group=None) -> torch.Tensor:
-    """(n_g, K) float64 per rank -> (world, n_g, K), block r from rank r."""
+    """(n_g, K) float64 per rank -> (world, n_g, K), block r from rank r, on the
+    device of sums64. Over NCCL the gather runs device to device; a gloo group
+    exchanges host copies (n_g (m+1+n) doubles per rank)."""
     world = dist.get_world_size(group)
     flat = sums64.contiguous().view(-1)
-    out = torch.empty((world * flat.numel(),), dtype=sums64.dtype, device=sums64.device)
-    dist.all_gather_into_tensor(out, flat, group=group)
+    host = sums64.is_cuda and dist.get_backend(group) == "gloo"
+    src = flat.cpu() if host else flat
+    out = torch.empty((world * flat.numel(),), dtype=sums64.dtype, device=src.device)
+    dist.all_gather_into_tensor(out, src, group=group)
+    if host:
+        out = out.to(sums64.device)
     return out.view((world,) + tuple(sums64.shape))
 
 
