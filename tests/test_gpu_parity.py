@@ -37,6 +37,9 @@ CASES = {
     # TMA stores (float32) and the buffered guarded stores (bf16)
     "box_partial_f32_dg40": _custom("box_f32_dg40", 301, 160, 4, 5, 4, synth.F32),
     "box_partial_bf16_dg40": _custom("box_bf16_dg40", 301, 160, 4, 5, 4, synth.BF16),
+    # one channel per group (d_g = 1): every channel its own coefficients
+    "dg1_f32": _custom("dg1_f32", 45, 16, 16, 5, 4, synth.F32),
+    "dg1_bf16": _custom("dg1_bf16", 45, 16, 16, 5, 4, synth.BF16),
     "deg_3_2": _custom("deg_3_2", 100, 384, 4, 3, 2, synth.BF16),
     "deg_0_0": _custom("deg_0_0", 60, 64, 2, 0, 0, synth.F32),
     "deg_8_8": _custom("deg_8_8", 60, 64, 4, 8, 8, synth.F32, x_kind=synth.KIND_NORMAL,
@@ -101,7 +104,8 @@ def test_fast_path_is_taken_where_expected():
         args = (w.rows, 1, w.d, w.n_g, w.m, w.n, w.dtype)
         assert grk.grkan_forward_path(t, t, *args) == 1, name
         assert grk.grkan_backward_path(t, t, t, *args) == 1, name
-    for name in ("odd_f32_dg10", "odd_bf16_dg6", "deg_3_2", "deg_0_0", "deg_5_0", "deg_2_6"):
+    for name in ("odd_f32_dg10", "odd_bf16_dg6", "deg_3_2", "deg_0_0", "deg_5_0", "deg_2_6",
+                 "dg1_f32", "dg1_bf16"):
         w = CASES[name]
         t = torch.empty((w.rows, w.d), dtype=torch.float32, device="cuda")
         assert grk.grkan_backward_path(t, t, t, w.rows, 1, w.d, w.n_g, w.m, w.n, w.dtype) == 0
