@@ -436,6 +436,7 @@ def main():
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
+    grads_warm = torch.cat([dA.flatten(), dB.flatten()]).clone()
 
     # timed region: exactly K steps between a barrier + synchronize on each side
     props = torch.cuda.get_device_properties(dev)
@@ -459,6 +460,14 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    # dA / dB after the last timed step against the copy taken after warm-up:
+    # the two-stage reduction gives the same bits every step
+    grads_last = torch.cat([dA.flatten(), dB.flatten()])
+    import hashlib
+    determinism = {
+        "dA_dB_identical_over_steps": bool(torch.equal(grads_warm, grads_last)),
+        "dA_dB_sha256_16": hashlib.sha256(
+            grads_last.cpu().numpy().tobytes()).hexdigest()[:16]}
     ms_total = t_start.elapsed_time(t_end)
     fwd_all = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_all = [e[1].elapsed_time(e[2]) for e in evs]
@@ -678,6 +687,7 @@ def main():
                 "api": "grkan_step_host (x, dy in; y, dx, dA, dB out; pinned host buffers)"},
         "fused_linear": linear,
         "per_config": per_config,
+        "determinism": determinism,
         "gpu_launches": args.steps * (3 + (1 if world > 1 else 0)),
         "clocks": clocks,
         "device_error": derr,
