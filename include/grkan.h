@@ -274,19 +274,18 @@ GRKAN_API grkan_status_t grkan_backward_noalloc(const void* x, const void* dy, c
  * data. sums64 (a DEVICE pointer, may be NULL) also receives the float64 sums
  * [n_g][m+1+n] that grkan_backward_merge would give, for a data-parallel merge
  * with grkan_merge_ranks. Asynchronous with respect to the host: the outputs are
- * complete once `stream` reaches the point of the call. The first call on a device creates
- * three streams and a few events that live until the process exits; calls are
- * serialised per device while they enqueue. */
+ * complete once `stream` reaches the point of the call. The first call on a
+ * device creates three streams and a few events that live until the process
+ * exits; calls are serialised per device while they enqueue. */
 GRKAN_API size_t grkan_step_host_scratch_bytes(int64_t B, int64_t N, int64_t d, int32_t n_g,
                                                int32_t m, int32_t n, grkan_dtype_t dtype,
                                                int64_t chunk_rows);
 GRKAN_API grkan_status_t grkan_step_host(const void* x_host, const void* dy_host, const float* a,
                                          const float* b, void* y_host, void* dx_host,
                                          float* dA_host, float* dB_host, double* sums64,
-                                         int64_t B, int64_t N,
-                                         int64_t d, int32_t n_g, int32_t m, int32_t n,
-                                         grkan_dtype_t dtype, void* scratch, size_t scratch_bytes,
-                                         int64_t chunk_rows, void* stream);
+                                         int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
+                                         int32_t n, grkan_dtype_t dtype, void* scratch,
+                                         size_t scratch_bytes, int64_t chunk_rows, void* stream);
 
 /* Which kernels a call with these arguments would run: 1 = TMA-pipelined
  * persistent kernels, 0 = generic grid-stride kernels, < 0 = invalid arguments
