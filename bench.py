@@ -261,7 +261,10 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(w.describe(), rows_per_step=rows),
+        "config": dict(w.describe(), global_batch=w.B * args.gpus, seq_len=w.N,
+                       parallelism="dp%d" % args.gpus,
+                       l2="host memory; each step a bounded sample of the workload",
+                       rows_per_step=rows),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
