@@ -46,7 +46,9 @@ def command(out=LIB, verbose=False, defines=()):
     knobs (GRK_BF16_BWD_WARPS, GRK_BF16_BWD_STAGES, GRK_FWD_WARPS, the store
     paths GRK_F32_FWD_STORE / GRK_BF16_FWD_STORE / GRK_F32_BWD_STORE /
     GRK_BF16_BWD_STORE, ... in csrc/grkan_tma.cuh; GRK_LIN_XFORM_WARPS in
-    csrc/grkan_linear.cuh; GRK_DG_STAGES in csrc/grkan_linear_bwd.cuh)."""
+    csrc/grkan_linear.cuh; GRK_DG_STAGES in csrc/grkan_linear_bwd.cuh;
+    GRK_LIN_QUAD, GRK_QD_RAW_STAGES, GRK_QD_A_STAGES, GRK_QD_EPI_BUFS in
+    csrc/grkan_linear_quad.cuh)."""
     cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
            "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
            *["-D" + d for d in defines], "-o", out, *SOURCES]

@@ -16,6 +16,7 @@
 #include "grkan_generic.cuh"
 #include "grkan_linear.cuh"
 #include "grkan_linear_bwd.cuh"
+#include "grkan_linear_quad.cuh"
 #include "grkan_merge.cuh"
 #include "grkan_tma.cuh"
 
@@ -644,6 +645,115 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// Clusters of four CTAs of the cluster fused forward that are resident at once
+// on the current device (a cluster needs four SMs of one GPC), looked up once
+// per device.
+cudaError_t quad_clusters(int* out) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+    *out = cached[dev];
+    return cudaSuccess;
+  }
+  namespace qd = grk::lin::qd;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(sms / 4 * 4), 1, 1);
+  cfg.blockDim = dim3(qd::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = qd::kAllocMax;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, qd::linear_fwd_quad, &cfg);
+  if (e != cudaSuccess) return e;
+  if (n < 1) n = 1;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  *out = n;
+  return cudaSuccess;
+}
+
+// Column tiling of the cluster fused forward: n_ct tiles of at most 2 x 512
+// outputs, split evenly between the two CTA pairs of a cluster, each pair's
+// share rounded up to 128 (two MMAs of at most 256, W boxes of 64 rows per CTA).
+void quad_cols(int64_t nout, int* np, int* n_ct) {
+  namespace qd = grk::lin::qd;
+  const long long ct = (nout + 2LL * qd::kNPMax - 1) / (2LL * qd::kNPMax);
+  const long long share = (nout + 2 * ct - 1) / (2 * ct);
+  *n_ct = (int)ct;
+  *np = (int)((share + 127) / 128 * 128);
+}
+
+// Whether grkan_linear_forward takes the cluster kernel. Its K steps cost about
+// the same time whatever the tile width (the activation path, not the tensor
+// cores, sets the pace), so it pays where a cluster's column tile is wide: one
+// tile of more than 512 outputs, or tiles whose pairs are 512 wide. Measured on
+// the KAT-B rows (100,864 x 3072): n_out 576 to 1024, 2048 and (d 768) 3072 are
+// faster than the one-CTA kernel; 512 and below, and 1536 (two tiles of 768),
+// are slower.
+bool use_linear_quad(const Plan& p, int64_t nout) {
+  if (!GRK_LIN_QUAD || p.d % grk::lin::qd::BK != 0 || nout <= 512) return false;
+  int np = 0, n_ct = 0;
+  quad_cols(nout, &np, &n_ct);
+  return n_ct == 1 || np == grk::lin::qd::kNPMax;
+}
+
+// The cluster fused forward: d a multiple of its K step (64); the plan, the
+// pointers and the other shapes are checked by the caller.
+cudaError_t launch_linear_quad(const void* x, const void* W, void* out, const Plan& p,
+                               int64_t nout, const float* a, const float* b, const float* bias,
+                               cudaStream_t st) {
+  namespace qd = grk::lin::qd;
+  CUtensorMap mx, mw, mo;
+  if (!make_map_bf16(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, qd::BK, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mw, W, (uint64_t)p.d, (uint64_t)nout, qd::BK, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mo, out, (uint64_t)nout, (uint64_t)p.rows, 64, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  qd::QGeom g;
+  g.rows = p.rows;
+  g.d = (int)p.d;
+  g.nout = (int)nout;
+  g.dg = (int)p.dg;
+  g.n_g = p.n_g;
+  g.kt = (int)(p.d / qd::BK);
+  quad_cols(nout, &g.np, &g.n_ct);
+  g.n1 = g.np < 256 ? g.np : 256;
+  g.n2 = g.np - g.n1;
+  g.n_tiles = ((p.rows + 2 * qd::BM - 1) / (2 * qd::BM)) * g.n_ct;
+  g.ws = qd::Layout::w_stages(g.np);
+  cudaError_t e = grk::ensure_smem<qd::linear_fwd_quad>(qd::kAllocMax);
+  int clusters = 0;
+  if (e == cudaSuccess) e = quad_clusters(&clusters);
+  if (e != cudaSuccess) return e;
+  if ((long long)clusters > g.n_tiles) clusters = (int)g.n_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(4 * clusters), 1, 1);
+  cfg.blockDim = dim3(qd::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = qd::Layout::alloc(g.np);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qd::linear_fwd_quad, mx, mw, mo, a, b, bias, g);
+}
+
 }  // namespace
 
 grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* b, const void* W,
@@ -655,7 +765,7 @@ grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* 
   if (s != GRKAN_OK) return s;
   if (p.dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
   if (p.m != 5 || p.n != 4) return GRKAN_ERR_DEGREE;
-  if (nout < 0 || p.d % grk::lin::BK != 0 || p.dg % 8 != 0 || nout % 8 != 0 ||
+  if (nout < 0 || p.d == 0 || p.d % grk::lin::BK != 0 || p.dg % 8 != 0 || nout % 8 != 0 ||
       p.rows > 0x7fffffffLL || nout > 0x7fffffffLL)
     return GRKAN_ERR_SHAPE;
   if (p.rows == 0 || nout == 0) return GRKAN_OK;
@@ -667,6 +777,9 @@ grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* 
   const size_t obytes = (size_t)p.rows * (size_t)nout * 2;
   if (overlaps(out, obytes, x, xbytes) || overlaps(out, obytes, W, wbytes)) return GRKAN_ERR_ALIAS;
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
+  if (use_linear_quad(p, nout))
+    return cuda_status(launch_linear_quad(x, W, out, p, nout, a, b, bias, (cudaStream_t)stream),
+                       "grkan_linear_forward launch");
   CUtensorMap mx, mw, mo;
   if (!make_map_bf16(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, grk::lin::BK, grk::lin::BM,
                      CU_TENSOR_MAP_SWIZZLE_64B) ||

@@ -147,8 +147,9 @@ GRKAN_API grkan_status_t grkan_forward_backward(const void* x, const void* dy, c
  * row-major, overwritten. y is rounded to bf16 before the product, as when
  * grkan_forward's output feeds a bf16 matrix multiply; the sum is float32.
  * Requires dtype GRKAN_BF16 (else GRKAN_ERR_DTYPE), (m, n) = (5, 4) (else
- * GRKAN_ERR_DEGREE), d % 32 == 0, d_g % 8 == 0, nout % 8 == 0 and 16-byte
- * aligned x, W, out (else GRKAN_ERR_SHAPE); out may not overlap x or W. */
+ * GRKAN_ERR_DEGREE), d > 0, d % 32 == 0, d_g % 8 == 0, nout % 8 == 0 and
+ * 16-byte aligned x, W, out (else GRKAN_ERR_SHAPE); out may not overlap x or W.
+ * B*N == 0 or nout == 0: nothing to do. */
 GRKAN_API grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* b,
                                               const void* W, const float* bias, void* out,
                                               int64_t B, int64_t N, int64_t d, int32_t n_g,

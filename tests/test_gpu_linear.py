@@ -1,9 +1,11 @@
 """GR-KAN fused into the following linear layer (grkan_linear_forward) against
 the fp64 oracle's activation times the weight in fp64, and against the same
-product taken from the library's own forward output. Shapes span several
-128-row and 256-column tiles, a ragged last tile in both, more K steps than the
-kernel's four-stage ring, groups that straddle a 64-channel K step, bias and no
-bias."""
+product taken from the library's own forward output. The shapes reach both
+kernels behind the call (one CTA per 128 x 512 tile for n_out up to 512, CTA
+clusters of four for wider outputs) and span several row and column tiles, a
+ragged last tile in both, more K steps than any ring has stages, more tiles than
+resident clusters, groups that straddle a 64-channel K step, bias and no bias.
+The output is written inside its region only."""
 import numpy as np
 import pytest
 import torch
@@ -50,6 +52,11 @@ def _reference(w, x, a, b, wt, bias):
     (130, 160, 20, 520, True),    # d_g 8 (many groups per K step), n_out just past a tile
     (300, 1536, 8, 384, True),    # second half 128 wide (narrower MMA)
     (200, 512, 8, 296, False),    # second half 40 wide: MMA width 48, store clipped at 296
+    (20000, 512, 8, 768, True),   # more 256-row tiles than resident CTAs: persistent walk
+    (700, 256, 4, 1536, False),   # n_out past 1024: two column tiles of a cluster
+    (600, 1024, 16, 2048, True),  # two column tiles of 1024
+    (300, 768, 8, 3072, True),    # the KAT second-linear's transpose: three column tiles
+    (100, 512, 8, 640, False),    # one ragged 256-row tile: half of it past the last row
 ])
 def test_fused_linear_matches_oracle(rows, d, n_g, nout, with_bias):
     w, x, a, b, wt, bias = _case(rows, d, n_g, nout)
@@ -91,3 +98,27 @@ def test_fused_linear_rejects_unsupported():
                                     grk.BF16) == 2  # d % 32
     assert grk.grkan_linear_forward(t, f, f, t, None, t, 0, 1, 64, 8, 5, 4, 64,
                                     grk.BF16) == 0  # empty: nothing to do
+    assert grk.grkan_linear_forward(t, f, f, t, None, t, 1, 1, 0, 8, 5, 4, 64,
+                                    grk.BF16) == 2  # d == 0
+
+
+@pytest.mark.parametrize("rows,d,nout", [(333, 512, 296), (333, 512, 768), (77, 768, 2048)])
+def test_fused_linear_writes_only_its_output(rows, d, nout):
+    """out sits between sentinel bytes; both kernels' clipped TMA stores (ragged
+    rows and columns) leave them untouched."""
+    n_g = 8
+    w, x, a, b, wt, bias = _case(rows, d, n_g, nout)
+    guard = 4096
+    nb = rows * nout * 2
+    buf = torch.full((guard + nb + guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    out = buf[guard:guard + nb].view(torch.bfloat16).view(rows, nout)
+    tx, tw = to_torch(x), to_torch(wt)
+    ta, tb = torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()
+    assert grk.grkan_linear_forward(tx, ta, tb, tw, None, out, rows, 1, d, n_g, 5, 4, nout,
+                                    grk.BF16) == 0
+    torch.cuda.synchronize()
+    host = buf.cpu().numpy()
+    assert np.all(host[:guard] == 0xA5) and np.all(host[guard + nb:] == 0xA5)
+    ref = grk.linear_forward(tx, ta, tb, n_g, tw, None)
+    assert torch.equal(out, ref)
+    assert grk.grkan_device_error()[1] == 0
