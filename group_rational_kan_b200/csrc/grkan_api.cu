@@ -645,10 +645,10 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-// Clusters of four CTAs of the cluster fused forward that are resident at once
-// on the current device (a cluster needs four SMs of one GPC), looked up once
-// per device.
-cudaError_t quad_clusters(int* out) {
+// Clusters of `size` CTAs of `kernel` (with `smem` bytes of dynamic shared
+// memory) that are resident at once on the current device, looked up once per
+// device (for the one kernel that asks: the cluster fused forward).
+cudaError_t resident_clusters(const void* kernel, int size, int threads, unsigned smem, int* out) {
   static std::mutex mu;
   static int cached[64] = {};
   int dev = 0;
@@ -659,23 +659,22 @@ cudaError_t quad_clusters(int* out) {
     *out = cached[dev];
     return cudaSuccess;
   }
-  namespace qd = grk::lin::qd;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(sms / 4 * 4), 1, 1);
-  cfg.blockDim = dim3(qd::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = qd::kAllocMax;
+  cfg.gridDim = dim3((unsigned)(sms / size * size), 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.x = (unsigned)size;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, qd::linear_fwd_quad, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
   if (e != cudaSuccess) return e;
   if (n < 1) n = 1;
   if (dev >= 0 && dev < 64) cached[dev] = n;
@@ -702,7 +701,9 @@ void quad_cols(int64_t nout, int* np, int* n_ct) {
 // faster than the one-CTA kernel; 512 and below, and 1536 (two tiles of 768),
 // are slower.
 bool use_linear_quad(const Plan& p, int64_t nout) {
-  if (!GRK_LIN_QUAD || p.d % grk::lin::qd::BK != 0 || nout <= 512) return false;
+  if (!GRK_LIN_QUAD || p.d % grk::lin::qd::BK != 0) return false;
+  if (GRK_LIN_QUAD == 2) return true;
+  if (nout <= 512) return false;
   int np = 0, n_ct = 0;
   quad_cols(nout, &np, &n_ct);
   return n_ct == 1 || np == grk::lin::qd::kNPMax;
@@ -736,7 +737,9 @@ cudaError_t launch_linear_quad(const void* x, const void* W, void* out, const Pl
   g.ws = qd::Layout::w_stages(g.np);
   cudaError_t e = grk::ensure_smem<qd::linear_fwd_quad>(qd::kAllocMax);
   int clusters = 0;
-  if (e == cudaSuccess) e = quad_clusters(&clusters);
+  if (e == cudaSuccess)
+    e = resident_clusters(reinterpret_cast<const void*>(qd::linear_fwd_quad), 4, qd::kThreads,
+                          qd::kAllocMax, &clusters);
   if (e != cudaSuccess) return e;
   if ((long long)clusters > g.n_tiles) clusters = (int)g.n_tiles;
   cudaLaunchConfig_t cfg = {};

@@ -46,7 +46,8 @@
 #include "grkan_linear_bwd.cuh"
 
 // 1: grkan_linear_forward takes this kernel for the shapes where it is the
-// faster of the two (use_linear_quad in grkan_api.cu); 0: never.
+// faster of the two (use_linear_quad in grkan_api.cu); 2: whenever d is a
+// multiple of 64; 0: never.
 #ifndef GRK_LIN_QUAD
 #define GRK_LIN_QUAD 1
 #endif
@@ -69,13 +70,13 @@ constexpr int BK = 64;           // K per stage: one 128-byte swizzle row of bf1
 // Ring depths and epilogue staging buffers per warp (launch-shape knobs; the
 // W ring takes what shared memory is left).
 #ifndef GRK_QD_RAW_STAGES
-#define GRK_QD_RAW_STAGES 3
+#define GRK_QD_RAW_STAGES 2
 #endif
 #ifndef GRK_QD_A_STAGES
-#define GRK_QD_A_STAGES 4
+#define GRK_QD_A_STAGES 5
 #endif
 #ifndef GRK_QD_EPI_BUFS
-#define GRK_QD_EPI_BUFS 2
+#define GRK_QD_EPI_BUFS 1
 #endif
 constexpr int kRawStages = GRK_QD_RAW_STAGES;
 constexpr int kAStages = GRK_QD_A_STAGES;
