@@ -646,17 +646,18 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
 }
 
 // Clusters of `size` CTAs of `kernel` (with `smem` bytes of dynamic shared
-// memory) that are resident at once on the current device, looked up once per
-// device (for the one kernel that asks: the cluster fused forward).
+// memory) that are resident at once on the current device (0 if none fits),
+// looked up once per device (for the one kernel that asks: the cluster fused
+// forward).
 cudaError_t resident_clusters(const void* kernel, int size, int threads, unsigned smem, int* out) {
   static std::mutex mu;
-  static int cached[64] = {};
+  static int cached[64];  // clusters + 1 once looked up
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
   if (dev >= 0 && dev < 64 && cached[dev] > 0) {
-    *out = cached[dev];
+    *out = cached[dev] - 1;
     return cudaSuccess;
   }
   int sms = 0;
@@ -676,8 +677,8 @@ cudaError_t resident_clusters(const void* kernel, int size, int threads, unsigne
   int n = 0;
   e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
   if (e != cudaSuccess) return e;
-  if (n < 1) n = 1;
-  if (dev >= 0 && dev < 64) cached[dev] = n;
+  if (n < 0) n = 0;
+  if (dev >= 0 && dev < 64) cached[dev] = n + 1;
   *out = n;
   return cudaSuccess;
 }
@@ -710,7 +711,9 @@ bool use_linear_quad(const Plan& p, int64_t nout) {
 }
 
 // The cluster fused forward: d a multiple of its K step (64); the plan, the
-// pointers and the other shapes are checked by the caller.
+// pointers and the other shapes are checked by the caller. Returns
+// cudaErrorNotSupported, having launched nothing, when no cluster of four fits
+// on the device.
 cudaError_t launch_linear_quad(const void* x, const void* W, void* out, const Plan& p,
                                int64_t nout, const float* a, const float* b, const float* bias,
                                cudaStream_t st) {
@@ -736,11 +739,14 @@ cudaError_t launch_linear_quad(const void* x, const void* W, void* out, const Pl
   g.n_tiles = ((p.rows + 2 * qd::BM - 1) / (2 * qd::BM)) * g.n_ct;
   g.ws = qd::Layout::w_stages(g.np);
   cudaError_t e = grk::ensure_smem<qd::linear_fwd_quad>(qd::kAllocMax);
-  int clusters = 0;
-  if (e == cudaSuccess)
-    e = resident_clusters(reinterpret_cast<const void*>(qd::linear_fwd_quad), 4, qd::kThreads,
-                          qd::kAllocMax, &clusters);
   if (e != cudaSuccess) return e;
+  int clusters = 0;
+  if (resident_clusters(reinterpret_cast<const void*>(qd::linear_fwd_quad), 4, qd::kThreads,
+                        qd::kAllocMax, &clusters) != cudaSuccess) {
+    (void)cudaGetLastError();  // the query failed: no cluster can be placed
+    return cudaErrorNotSupported;
+  }
+  if (clusters < 1) return cudaErrorNotSupported;
   if ((long long)clusters > g.n_tiles) clusters = (int)g.n_tiles;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(4 * clusters), 1, 1);
@@ -780,9 +786,12 @@ grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* 
   const size_t obytes = (size_t)p.rows * (size_t)nout * 2;
   if (overlaps(out, obytes, x, xbytes) || overlaps(out, obytes, W, wbytes)) return GRKAN_ERR_ALIAS;
   if (!is_sm100()) return GRKAN_ERR_DEVICE;
-  if (use_linear_quad(p, nout))
-    return cuda_status(launch_linear_quad(x, W, out, p, nout, a, b, bias, (cudaStream_t)stream),
-                       "grkan_linear_forward launch");
+  if (use_linear_quad(p, nout)) {
+    const cudaError_t eq =
+        launch_linear_quad(x, W, out, p, nout, a, b, bias, (cudaStream_t)stream);
+    // no cluster of four fits on this device: the one-CTA kernel below
+    if (eq != cudaErrorNotSupported) return cuda_status(eq, "grkan_linear_forward launch");
+  }
   CUtensorMap mx, mw, mo;
   if (!make_map_bf16(&mx, x, (uint64_t)p.d, (uint64_t)p.rows, grk::lin::BK, grk::lin::BM,
                      CU_TENSOR_MAP_SWIZZLE_64B) ||
