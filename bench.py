@@ -71,6 +71,17 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
 
 
+def tensor_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s) for a kernel timed alone: the
+    measured burst cuBLAS figure, else the fallback measurement."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return 1590.0, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+
+
 def measured_traffic(w):
     """DRAM bytes per backward launch from the committed ncu summary, scaled by
     elements; None unless the summary covers this workload and the kernel
@@ -531,11 +542,26 @@ def main():
             return t0.elapsed_time(t1) / k
 
         fl = 2.0 * B * N * d * nout
-        f_ms, u_ms = timed(lin_fused), timed(lin_unfused)
+        tpeak, tsrc = tensor_peak()
+
+        def tensor_roofline(ms):
+            ach = fl / (ms * 1e-3) / 1e12
+            return {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": ach / tpeak, "peak_source": tsrc,
+                    "flops_per_launch": fl}
+
+        # alternated three times, medians
+        ff, uf = [], []
+        for _ in range(3):
+            ff.append(timed(lin_fused))
+            uf.append(timed(lin_unfused))
+        f_ms, u_ms = sorted(ff)[1], sorted(uf)[1]
         linear = {"nout": nout, "fused_ms": f_ms, "unfused_ms": u_ms,
                   "fused_TFLOP/s": fl / (f_ms * 1e-3) / 1e12,
+                  "roofline": tensor_roofline(f_ms),
                   "note": "grkan_linear_forward vs grkan_forward + torch.matmul (cuBLAS), "
-                          "no bias; not part of the timed step"}
+                          "no bias; not part of the timed step; the kernel behind the call is "
+                          "chosen by shape (n_out > 512: clusters of four CTAs)"}
 
         # its backward: dy = dout W on the tensor cores with the GR-KAN backward as
         # the epilogue, against torch.matmul (cuBLAS, bf16 dy) + grkan_backward;
@@ -562,6 +588,7 @@ def main():
         linear["backward"] = {
             "fused_ms": fb_ms, "unfused_ms": ub_ms,
             "fused_TFLOP/s": fl / (fb_ms * 1e-3) / 1e12,
+            "roofline": tensor_roofline(fb_ms),
             "note": "grkan_linear_backward (dout W + GR-KAN backward epilogue, CTA pairs) vs "
                     "torch.matmul (cuBLAS) + grkan_backward; weight gradient not included"}
         del Wl, outl, dout, dyl, wsl

@@ -1,7 +1,8 @@
 """bench.py on the GPU, on a small slice of the KAT-B workload: one JSON line
 with the keys and units the measurement contract asks for, a roofline and an
-ALU roofline for the backward kernel, the end-to-end leg through host buffers,
-the determinism check, and per-workload timings."""
+ALU roofline for the backward kernel, tensor rooflines for the fused linear
+layer, the end-to-end leg through host buffers, the determinism check, and
+per-workload timings."""
 import json
 import os
 import subprocess
@@ -41,5 +42,11 @@ def test_bench_json_line():
     assert d["determinism"]["dA_dB_identical_over_steps"] is True
     assert d["clocks"] is None or d["clocks"]["samples"] >= 1
     assert [c["workload"] for c in d["per_config"]] == ["kat_t", "stress_ng64"]
-    assert d["fused_linear"]["nout"] == 512
+    fl = d["fused_linear"]
+    assert fl["nout"] == 512
+    for part in (fl, fl["backward"]):
+        r = part["roofline"]
+        assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and 0 < r["frac"] < 1.5
+        assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+        assert r["flops_per_launch"] == 2.0 * 4000 * 3072 * 512
     assert d["device_error"] == 0
