@@ -122,3 +122,24 @@ def test_fused_linear_writes_only_its_output(rows, d, nout):
     ref = grk.linear_forward(tx, ta, tb, n_g, tw, None)
     assert torch.equal(out, ref)
     assert grk.grkan_device_error()[1] == 0
+
+
+@pytest.mark.parametrize("rows,d,with_bias", [(1000, 3072, True), (333, 512, False)])
+def test_fused_linear_kernels_agree(rows, d, with_bias):
+    """n_out = 768 takes the cluster kernel, n_out <= 512 the one-CTA kernel. Every
+    output element is the same bf16 y row times one W row, summed over K in the
+    same 16-wide slices in the same order, so the 768 columns equal, bit for bit,
+    the one-CTA kernel's results for the column slices [0, 512) and [512, 768)."""
+    n_g, nout = 8, 768
+    w, x, a, b, wt, bias = _case(rows, d, n_g, nout)
+    tx, tw = to_torch(x), to_torch(wt)
+    ta, tb = torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()
+    tbias = torch.from_numpy(bias).cuda() if with_bias else None
+    full = grk.linear_forward(tx, ta, tb, n_g, tw, tbias)
+    lo = grk.linear_forward(tx, ta, tb, n_g, tw[:512].contiguous(),
+                            tbias[:512].contiguous() if with_bias else None)
+    hi = grk.linear_forward(tx, ta, tb, n_g, tw[512:].contiguous(),
+                            tbias[512:].contiguous() if with_bias else None)
+    torch.cuda.synchronize()
+    assert torch.equal(full[:, :512], lo) and torch.equal(full[:, 512:], hi)
+    assert grk.grkan_device_error()[1] == 0
