@@ -32,14 +32,17 @@
 //                in all four CTAs with multicast commits. In the other CTA lane
 //                0 tells the leader when its A stage is complete;
 //   warp 2       lane 0 loads the W ring;
-//   warps 3..18  activate one 16-byte chunk each per K step: raw slot ->
+//   8 warps      activate two 16-byte chunks each per K step: raw slot ->
 //                registers -> activation -> this CTA's half of the A stage. The
-//                last of the sixteen warps to finish a stage (a shared counter)
+//                last of the eight warps to finish a stage (a shared counter)
 //                copies the half into the partner's stage and marks it ready;
-//   warps 19..22 the epilogue: read the accumulator (one TMEM lane quarter
+//   4 warps      the epilogue: read the accumulator (one TMEM lane quarter
 //                each), add the bias, convert to bf16 and write the tile with
 //                TMA stores through 128-byte-swizzled staging buffers, then free
 //                the accumulator for the next tile.
+// Warp w runs on scheduler w % 4. The transform warps are placed off warp 1's
+// scheduler: they wake on the same stage releases that the MMA issuer waits
+// for, and sharing its scheduler slowed the issue of the next K step's MMAs.
 // Every wait is bounded (device error word), and TMEM is freed on every path.
 #pragma once
 
@@ -83,20 +86,36 @@ constexpr int kAStages = GRK_QD_A_STAGES;
 constexpr int kEpiBufs = GRK_QD_EPI_BUFS;
 constexpr int kWStagesMax = 6;
 constexpr int kNPMax = 512;      // outputs per pair: the TMEM columns
-constexpr int kXformWarps = 16;
+constexpr int kXformWarps = 8;
 constexpr int kEpiWarps = 4;
-constexpr int kXformWarp0 = 3;  // warps 0..2: x producer, MMA / forwarder, W producer
-constexpr int kEpiWarp0 = kXformWarp0 + kXformWarps;
-constexpr int kWarps = kEpiWarp0 + kEpiWarps;
+// Warp roles: 0 x producer, 1 MMA issue (leader) or forwarder, 2 W producer;
+// transform warps 4, 8, 12, 6, 10, 14, 3, 7 (in their index order); epilogue
+// warps 16, 5, 18, 15 (an epilogue warp reads TMEM lane quarter warp % 4, so
+// these cover the 128 lanes); warps 9, 11, 13, 17, 19 idle. Warp 1's scheduler
+// (warps 1, 5, 9, ...) holds no transform warp.
+constexpr int kWarps = 20;
 constexpr int kThreads = kWarps * 32;
-// an epilogue warp reads TMEM lane quarter warp % 4, so four consecutive warps
-// cover the 128 lanes
-static_assert(kEpiWarps == 4, "one epilogue warp per TMEM lane quarter");
+__device__ __forceinline__ int xform_index(int w) {
+  switch (w) {
+    case 4: return 0;
+    case 8: return 1;
+    case 12: return 2;
+    case 6: return 3;
+    case 10: return 4;
+    case 14: return 5;
+    case 3: return 6;
+    case 7: return 7;
+    default: return -1;
+  }
+}
+__device__ __forceinline__ int epi_index(int w) {
+  return w == 16 ? 0 : w == 5 ? 1 : w == 18 ? 2 : w == 15 ? 3 : -1;
+}
 constexpr unsigned kRaw = 64 * BK * 2;            // 8 KiB: the CTA's 64 raw rows
 constexpr unsigned kATile = 2 * kRaw;             // 16 KiB: the CTA's 128 operand rows
 constexpr unsigned kWBox = 64 * BK * 2;           // 8 KiB: 64 W rows
 constexpr unsigned kEpiBuf = 32 * 64 * 2;         // 4 KiB: 32 rows x 64 outputs
-static_assert(kXformWarps * 32 == 64 * (BK / 8), "one 16-byte chunk per transform thread");
+static_assert(kXformWarps * 32 * 2 == 64 * (BK / 8), "two 16-byte chunks per transform thread");
 static_assert(kEpiBufs == 1 || kEpiBufs == 2, "one or two staging buffers per epilogue warp");
 
 // Shared memory, from a 1024-byte aligned base: raw ring, A ring, epilogue
@@ -422,13 +441,14 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
         mbar_arrive_release_cluster(lead_ready0 + 8u * (uint32_t)ra.s);
       }
     }
-  } else if (warp < kEpiWarp0) {
-    // ---- activation: one 16-byte chunk per thread and K step, into this CTA's
-    // half of the A stage ------------------------------------------------------------------
-    const int t = threadIdx.x - 32 * kXformWarp0;  // 0 .. 511
-    const int rr = t >> 3;  // row of the CTA's 64 raw rows
+  } else if (xform_index(warp) >= 0) {
+    // ---- activation: two 16-byte chunks per thread and K step (rows rr and
+    // rr + 32), into this CTA's half of the A stage -----------------------------------------
+    const int t = xform_index(warp) * 32 + lane;  // 0 .. 255
+    const int rr = t >> 3;  // rows rr and rr + 32 of the CTA's 64 raw rows
     const int j = t & 7;    // logical 16-byte chunk (8 channels) of the 128-byte row
-    const uint32_t sw = (uint32_t)(j ^ (rr & 7)) << 4;  // 128-byte swizzle (8-row atoms)
+    // 128-byte swizzle (8-row atoms): rows rr and rr + 32 share the xor pattern
+    const uint32_t sw = (uint32_t)(j ^ (rr & 7)) << 4;
     const uint32_t raw_off = (uint32_t)rr * 128u + sw;
     const uint32_t a_off = ((uint32_t)p * 64u + (uint32_t)rr) * 128u + sw;
     const uint32_t part_a0 = peer_addr(a_addr(0), partner) + p * kRaw;
@@ -451,7 +471,9 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
           ok = false;
           break;
         }
-        uint4 v = *reinterpret_cast<const uint4*>(smem + (size_t)sx * kRaw + raw_off);
+        const unsigned char* raw = smem + (size_t)sx * kRaw + raw_off;
+        uint4 v = *reinterpret_cast<const uint4*>(raw);
+        uint4 v2 = *reinterpret_cast<const uint4*>(raw + 32u * 128u);
         __syncwarp();
         if (lane == 0) mbar_arrive(xempty_bar(sx));  // the slot is read
         while (ch >= gend) {  // a chunk lies in one group (d_g % 8 == 0)
@@ -466,6 +488,10 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
         v.y = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.y)));
         v.z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.z)));
         v.w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v.w)));
+        v2.x = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v2.x)));
+        v2.y = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v2.y)));
+        v2.z = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v2.z)));
+        v2.w = f2_to_bf16x2(fwd_pair(c, bf16x2_to_f2(v2.w)));
         // the A stage is free in this CTA and the partner once both pairs' MMAs
         // of its previous use are done
         got = mbar_wait_sleep(aempty_bar(sa), ra.ph ^ 1u);
@@ -474,7 +500,9 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
           ok = false;
           break;
         }
-        *reinterpret_cast<uint4*>(smem + Layout::kAOff + (size_t)sa * kATile + a_off) = v;
+        unsigned char* at = smem + Layout::kAOff + (size_t)sa * kATile + a_off;
+        *reinterpret_cast<uint4*>(at) = v;
+        *reinterpret_cast<uint4*>(at + 32u * 128u) = v2;
         fence_proxy_async_smem();  // before the copy's and the tensor cores' reads
         __syncwarp();
         if (lane == 0) {
@@ -498,10 +526,10 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
     if (t == 0)
       for (long long u = kc > A ? kc - A : 0; u < kc; ++u)
         if (!mbar_wait(aready_bar((int)(u % A)), (uint32_t)(u / A) & 1u)) report(kErrDrainWait);
-  } else {
+  } else if (epi_index(warp) >= 0) {
     // ---- epilogue: accumulator -> bf16 -> TMA stores --------------------------------------
     const int q = warp & 3;  // TMEM lane quarter: rows 32 q .. 32 q + 31 of the CTA's 128
-    const int e = warp - kEpiWarp0;
+    const int e = epi_index(warp);
     unsigned char* stg = smem + Layout::kStgOff + (size_t)e * kEpiBufs * kEpiBuf;
     const uint32_t stg_a = sbase + Layout::kStgOff + (uint32_t)e * (uint32_t)kEpiBufs * kEpiBuf;
     const uint32_t lead_acce = peer_addr(acce_bar, lead);
