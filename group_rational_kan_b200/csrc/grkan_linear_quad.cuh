@@ -70,19 +70,22 @@ using dg::umma2_bf16;
 
 constexpr int BM = 128;          // rows per CTA; a pair covers 256 (UMMA M)
 constexpr int BK = 64;           // K per stage: one 128-byte swizzle row of bf16
-// Ring depths and epilogue staging buffers per warp (launch-shape knobs; the
-// W ring takes what shared memory is left).
+// Ring depths and epilogue staging buffers per warp (launch-shape knobs). The
+// operand ring is GRK_QD_A_STAGES deep for pair tiles of up to 384 outputs and
+// 5 deep for 512 (whose W stages are larger); the W ring takes what shared
+// memory is left.
 #ifndef GRK_QD_RAW_STAGES
 #define GRK_QD_RAW_STAGES 2
 #endif
 #ifndef GRK_QD_A_STAGES
-#define GRK_QD_A_STAGES 5
+#define GRK_QD_A_STAGES 7
 #endif
 #ifndef GRK_QD_EPI_BUFS
 #define GRK_QD_EPI_BUFS 1
 #endif
 constexpr int kRawStages = GRK_QD_RAW_STAGES;
-constexpr int kAStages = GRK_QD_A_STAGES;
+constexpr int kAStagesMax = GRK_QD_A_STAGES;
+static_assert(kAStagesMax >= 5, "the operand ring's depth at the widest tiles");
 constexpr int kEpiBufs = GRK_QD_EPI_BUFS;
 constexpr int kWStagesMax = 6;
 constexpr int kNPMax = 512;      // outputs per pair: the TMEM columns
@@ -120,31 +123,37 @@ static_assert(kEpiBufs == 1 || kEpiBufs == 2, "one or two staging buffers per ep
 
 // Shared memory, from a 1024-byte aligned base: raw ring, A ring, epilogue
 // staging, then the W ring (its stage size depends on NP, its depth is chosen
-// to fill what is left), the barriers, the TMEM slot and the coefficient table.
+// to fill what is left), the barriers, the TMEM slot, the per-A-stage counters
+// of finished transform warps and the coefficient table. Everything after the
+// raw ring depends on NP.
 struct Layout {
   static constexpr unsigned kAOff = kRawStages * kRaw;
-  static constexpr unsigned kStgOff = kAOff + kAStages * kATile;
-  static constexpr unsigned kWOff = kStgOff + kEpiWarps * kEpiBufs * kEpiBuf;
-  // xfull[R], xempty[R], aready[A], aempty[A], wfull[Wmax], wempty[Wmax], acc_full,
-  // acc_empty, done; then the TMEM slot, the per-A-stage counters of finished
-  // transform warps and the coefficient table
-  static constexpr unsigned kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kWStagesMax + 3;
-  static constexpr unsigned kTail = kNumBars * 8 + 16 + 4 * kAStages + 16 + coef_table_bytes<5, 4>();
+  // xfull[R], xempty[R], aready[Amax], aempty[Amax], wfull[Wmax], wempty[Wmax],
+  // acc_full, acc_empty, done
+  static constexpr unsigned kNumBars = 2 * kRawStages + 2 * kAStagesMax + 2 * kWStagesMax + 3;
+  static constexpr unsigned kTail = kNumBars * 8 + 16 + 4 * kAStagesMax + 16 + coef_table_bytes<5, 4>();
   static constexpr unsigned kMaxBytes = 232448 - 1024;  // the opt-in limit less the alignment slack
+  __host__ __device__ static constexpr int a_stages(int np) { return np > 384 ? 5 : kAStagesMax; }
+  __host__ __device__ static constexpr unsigned stg_off(int np) {
+    return kAOff + (unsigned)a_stages(np) * kATile;
+  }
+  __host__ __device__ static constexpr unsigned w_off(int np) {
+    return stg_off(np) + kEpiWarps * kEpiBufs * kEpiBuf;
+  }
   // bytes of a W stage (the CTA's NP / 2 rows) and the ring depth that fits
   __host__ __device__ static constexpr unsigned w_stage(int np) { return (unsigned)(np / 2) * BK * 2; }
   __host__ __device__ static constexpr int w_stages(int np) {
-    return (int)((kMaxBytes - kWOff - kTail) / w_stage(np)) < kWStagesMax
-               ? (int)((kMaxBytes - kWOff - kTail) / w_stage(np))
+    return (int)((kMaxBytes - w_off(np) - kTail) / w_stage(np)) < kWStagesMax
+               ? (int)((kMaxBytes - w_off(np) - kTail) / w_stage(np))
                : kWStagesMax;
   }
   __host__ __device__ static constexpr unsigned bar_off(int np) {
-    return kWOff + (unsigned)w_stages(np) * w_stage(np);
+    return w_off(np) + (unsigned)w_stages(np) * w_stage(np);
   }
   __host__ __device__ static constexpr unsigned tmem_slot(int np) { return bar_off(np) + kNumBars * 8; }
   __host__ __device__ static constexpr unsigned cnt_off(int np) { return (tmem_slot(np) + 4 + 15) / 16 * 16; }
   __host__ __device__ static constexpr unsigned tab_off(int np) {
-    return (cnt_off(np) + 4 * kAStages + 15) / 16 * 16;
+    return (cnt_off(np) + 4 * kAStagesMax + 15) / 16 * 16;
   }
   __host__ __device__ static constexpr unsigned alloc(int np) {
     return tab_off(np) + coef_table_bytes<5, 4>() + 1024;
@@ -159,8 +168,10 @@ constexpr unsigned kAllocMax =
         : (Layout::alloc(256) > Layout::alloc(384)
                ? (Layout::alloc(256) > Layout::alloc(512) ? Layout::alloc(256) : Layout::alloc(512))
                : (Layout::alloc(384) > Layout::alloc(512) ? Layout::alloc(384) : Layout::alloc(512)));
-static_assert(Layout::kWOff % 1024 == 0, "the W ring starts on a swizzle-atom boundary");
-static_assert(Layout::w_stages(kNPMax) >= 2, "two W stages at the widest tile");
+static_assert(Layout::w_off(128) % 1024 == 0 && Layout::w_off(512) % 1024 == 0,
+              "the W ring starts on a swizzle-atom boundary");
+static_assert(Layout::w_stages(kNPMax) >= 3 && Layout::w_stages(384) >= 3,
+              "three W stages at the widest tiles");
 static_assert(kAllocMax <= 232448, "shared memory per CTA");
 
 // Instruction descriptor: float32 accumulator, bf16 A and B, both K-major,
@@ -271,19 +282,21 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
   const uint32_t wbytes = Layout::w_stage(geom.np);  // this CTA's W rows of a K step
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + Layout::bar_off(geom.np);
-  constexpr int R = kRawStages, A = kAStages;
+  constexpr int R = kRawStages;
+  const int A = Layout::a_stages(geom.np);
   auto xfull_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
   auto xempty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(R + s); };
   auto aready_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + s); };
-  auto aempty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + A + s); };
-  auto wfull_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + 2 * A + s); };
-  auto wempty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + 2 * A + kWStagesMax + s); };
-  const uint32_t accf_bar = bar0 + 8u * (uint32_t)(2 * R + 2 * A + 2 * kWStagesMax);
+  constexpr int AM = kAStagesMax;
+  auto aempty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + AM + s); };
+  auto wfull_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + 2 * AM + s); };
+  auto wempty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * R + 2 * AM + kWStagesMax + s); };
+  const uint32_t accf_bar = bar0 + 8u * (uint32_t)(2 * R + 2 * AM + 2 * kWStagesMax);
   const uint32_t acce_bar = accf_bar + 8u;
   const uint32_t done_bar = accf_bar + 16u;
   auto raw_addr = [&](int s) { return sbase + (uint32_t)s * kRaw; };
   auto a_addr = [&](int s) { return sbase + Layout::kAOff + (uint32_t)s * kATile; };
-  auto w_addr = [&](int s) { return sbase + Layout::kWOff + (uint32_t)s * wbytes; };
+  auto w_addr = [&](int s) { return sbase + Layout::w_off(geom.np) + (uint32_t)s * wbytes; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Layout::tmem_slot(geom.np));
   unsigned* xcnt = reinterpret_cast<unsigned*>(smem + Layout::cnt_off(geom.np));
   float* ctab = reinterpret_cast<float*>(smem + Layout::tab_off(geom.np));
@@ -530,8 +543,9 @@ linear_fwd_quad(const __grid_constant__ CUtensorMap mx, const __grid_constant__ 
     // ---- epilogue: accumulator -> bf16 -> TMA stores --------------------------------------
     const int q = warp & 3;  // TMEM lane quarter: rows 32 q .. 32 q + 31 of the CTA's 128
     const int e = epi_index(warp);
-    unsigned char* stg = smem + Layout::kStgOff + (size_t)e * kEpiBufs * kEpiBuf;
-    const uint32_t stg_a = sbase + Layout::kStgOff + (uint32_t)e * (uint32_t)kEpiBufs * kEpiBuf;
+    const unsigned stg_off = Layout::stg_off(geom.np) + (unsigned)e * (unsigned)kEpiBufs * kEpiBuf;
+    unsigned char* stg = smem + stg_off;
+    const uint32_t stg_a = sbase + stg_off;
     const uint32_t lead_acce = peer_addr(acce_bar, lead);
     long long sc = 0;  // stores issued by this warp
     int i = 0;
