@@ -556,12 +556,13 @@ def main():
             ff.append(timed(lin_fused))
             uf.append(timed(lin_unfused))
         f_ms, u_ms = sorted(ff)[1], sorted(uf)[1]
+        path = grk.grkan_linear_forward_path(B, N, d, n_g, m, n, nout, dt)
         linear = {"nout": nout, "fused_ms": f_ms, "unfused_ms": u_ms,
                   "fused_TFLOP/s": fl / (f_ms * 1e-3) / 1e12,
                   "roofline": tensor_roofline(f_ms),
+                  "kernel": {1: "clusters of four CTAs", 0: "one CTA per tile"}.get(path, path),
                   "note": "grkan_linear_forward vs grkan_forward + torch.matmul (cuBLAS), "
-                          "no bias; not part of the timed step; the kernel behind the call is "
-                          "chosen by shape (n_out > 512: clusters of four CTAs)"}
+                          "no bias; not part of the timed step"}
 
         # its backward: dy = dout W on the tensor cores with the GR-KAN backward as
         # the epilogue, against torch.matmul (cuBLAS, bf16 dy) + grkan_backward;

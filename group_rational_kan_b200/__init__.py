@@ -19,7 +19,7 @@ __all__ = [
     "grkan_merge_ranks", "grkan_backward_noalloc", "NOALLOC_WORKSPACE_BYTES",
     "grkan_step_host", "grkan_step_host_scratch_bytes", "grkan_forward_backward",
     "grkan_backward_atomic", "ATOMIC_PER_ELEMENT", "ATOMIC_PER_BLOCK",
-    "grkan_linear_forward", "linear_forward",
+    "grkan_linear_forward", "grkan_linear_forward_path", "linear_forward",
     "grkan_linear_backward", "grkan_linear_backward_workspace_bytes", "linear_backward",
     "forward_backward",
     "grkan_forward_path", "grkan_backward_path", "grkan_device_error", "grkan_clear_device_error",
@@ -31,7 +31,7 @@ F32, BF16 = 0, 1
 FLAG_GENERIC = 1
 NOALLOC_WORKSPACE_BYTES = 4 << 20  # GRKAN_NOALLOC_WORKSPACE_BYTES
 DEVICE_ERROR_SELFTEST = 16  # GRKAN_DEVICE_ERROR_SELFTEST
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libgrkan_b200.so")
@@ -73,6 +73,7 @@ def _load():
         "grkan_merge_ranks": (S, [P, I32, P, P, I32, I32, I32, P]),
         "grkan_linear_forward": (S, [P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I64,
                                      ctypes.c_int, P]),
+        "grkan_linear_forward_path": (I32, [I64, I64, I64, I32, I32, I32, I64, ctypes.c_int]),
         "grkan_linear_backward_workspace_bytes": (SZ, [I64, I64, I64, I32, I32, I32, I64,
                                                        ctypes.c_int]),
         "grkan_linear_backward": (S, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I64,
@@ -95,13 +96,15 @@ def _load():
         "grkan_abi_version": (I32, []),
         "grkan_last_error": (ctypes.c_char_p, []),
     }
+    L.grkan_abi_version.restype = I32
+    L.grkan_abi_version.argtypes = []
+    if L.grkan_abi_version() != ABI_VERSION:
+        raise ImportError("libgrkan_b200.so ABI %d, binding expects %d" %
+                          (L.grkan_abi_version(), ABI_VERSION))
     for name, (res, args) in sig.items():
         f = getattr(L, name)
         f.restype = res
         f.argtypes = args
-    if L.grkan_abi_version() != ABI_VERSION:
-        raise ImportError("libgrkan_b200.so ABI %d, binding expects %d" %
-                          (L.grkan_abi_version(), ABI_VERSION))
     return L
 
 
@@ -194,6 +197,10 @@ ATOMIC_PER_BLOCK = 2
 def grkan_linear_forward(x, a, b, W, bias, out, B, N, d, n_g, m, n, nout, dtype, stream=None):
     return lib().grkan_linear_forward(_ptr(x), _ptr(a), _ptr(b), _ptr(W), _ptr(bias), _ptr(out),
                                       B, N, d, n_g, m, n, nout, dtype, _stream(stream))
+
+
+def grkan_linear_forward_path(B, N, d, n_g, m, n, nout, dtype):
+    return lib().grkan_linear_forward_path(B, N, d, n_g, m, n, nout, dtype)
 
 
 def linear_forward(x, a, b, n_g, W, bias=None, stream=None):

@@ -765,6 +765,29 @@ cudaError_t launch_linear_quad(const void* x, const void* W, void* out, const Pl
 
 }  // namespace
 
+namespace {
+
+// Shape checks of grkan_linear_forward (the plan is valid).
+grkan_status_t linear_fwd_shape(const Plan& p, int64_t nout) {
+  if (p.dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
+  if (p.m != 5 || p.n != 4) return GRKAN_ERR_DEGREE;
+  if (nout < 0 || p.d == 0 || p.d % grk::lin::BK != 0 || p.dg % 8 != 0 || nout % 8 != 0 ||
+      p.rows > 0x7fffffffLL || nout > 0x7fffffffLL)
+    return GRKAN_ERR_SHAPE;
+  return GRKAN_OK;
+}
+
+}  // namespace
+
+int32_t grkan_linear_forward_path(int64_t B, int64_t N, int64_t d, int32_t n_g, int32_t m,
+                                  int32_t n, int64_t nout, grkan_dtype_t dtype) {
+  Plan p;
+  grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
+  if (s == GRKAN_OK) s = linear_fwd_shape(p, nout);
+  if (s != GRKAN_OK) return -(int32_t)s;
+  return use_linear_quad(p, nout) ? 1 : 0;
+}
+
 grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* b, const void* W,
                                     const float* bias, void* out, int64_t B, int64_t N,
                                     int64_t d, int32_t n_g, int32_t m, int32_t n, int64_t nout,
@@ -772,11 +795,7 @@ grkan_status_t grkan_linear_forward(const void* x, const float* a, const float* 
   Plan p;
   grkan_status_t s = make_plan(B, N, d, n_g, m, n, dtype, &p);
   if (s != GRKAN_OK) return s;
-  if (p.dtype != GRKAN_BF16) return GRKAN_ERR_DTYPE;
-  if (p.m != 5 || p.n != 4) return GRKAN_ERR_DEGREE;
-  if (nout < 0 || p.d == 0 || p.d % grk::lin::BK != 0 || p.dg % 8 != 0 || nout % 8 != 0 ||
-      p.rows > 0x7fffffffLL || nout > 0x7fffffffLL)
-    return GRKAN_ERR_SHAPE;
+  if ((s = linear_fwd_shape(p, nout)) != GRKAN_OK) return s;
   if (p.rows == 0 || nout == 0) return GRKAN_OK;
   if (!x || !W || !out) return GRKAN_ERR_NULL;
   if ((s = check_coef_ptrs(p, a, b)) != GRKAN_OK) return s;

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(grk.library_path if os.path.exists(grk.library_path) else grk.lib()._name)
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert grk.grkan_abi_version() == grk.ABI_VERSION == 2
+    assert grk.grkan_abi_version() == grk.ABI_VERSION == 3
 
 
 def test_status_strings():
@@ -68,6 +68,29 @@ def test_path_selection():
     assert grk.grkan_forward_path(A, A, 2, 3, 12, 5, 5, 4, grk.F32) == -SHAPE
     assert grk.grkan_forward_path(A, A, 2, 3, 12, 3, 5, 4, 7) == -DTYPE
     assert grk.grkan_forward_path(A, A, 2, 3, 12, 3, 5, 4, grk.F32, flags=8) == -FLAGS
+
+
+def test_linear_forward_path():
+    """The fused linear forward's kernel by shape (no device needed): the cluster
+    kernel for n_out > 512 when one column tile or 512-wide pairs cover it and d is
+    a multiple of 64, the one-CTA kernel otherwise."""
+    p = grk.grkan_linear_forward_path
+    kat_b = (512, 197, 3072, 8, 5, 4)
+    assert p(*kat_b, 768, grk.BF16) == 1    # one tile, pairs of 384
+    assert p(*kat_b, 1024, grk.BF16) == 1   # one tile, pairs of 512
+    assert p(*kat_b, 576, grk.BF16) == 1
+    assert p(*kat_b, 512, grk.BF16) == 0    # one 512-column pass of the one-CTA kernel
+    assert p(*kat_b, 384, grk.BF16) == 0
+    assert p(*kat_b, 1536, grk.BF16) == 0   # two tiles with pairs of 384
+    assert p(*kat_b, 2048, grk.BF16) == 1   # two tiles with pairs of 512
+    assert p(512, 197, 768, 8, 5, 4, 3072, grk.BF16) == 1   # three tiles of 1024
+    assert p(2, 3, 160, 20, 5, 4, 768, grk.BF16) == 0       # d not a multiple of 64
+    assert p(0, 197, 3072, 8, 5, 4, 768, grk.BF16) == 1     # empty: the shape rule still holds
+    assert p(*kat_b, 768, grk.F32) == -DTYPE
+    assert p(512, 197, 3072, 8, 3, 3, 768, grk.BF16) == -DEGREE
+    assert p(*kat_b, 770, grk.BF16) == -SHAPE              # n_out % 8
+    assert p(512, 197, 48, 6, 5, 4, 768, grk.BF16) == -SHAPE  # d % 32
+    assert p(1, 1, 0, 8, 5, 4, 64, grk.BF16) == -SHAPE     # d == 0
 
 
 def test_argument_errors_need_no_gpu():

@@ -43,7 +43,7 @@ def test_bench_json_line():
     assert d["clocks"] is None or d["clocks"]["samples"] >= 1
     assert [c["workload"] for c in d["per_config"]] == ["kat_t", "stress_ng64"]
     fl = d["fused_linear"]
-    assert fl["nout"] == 512
+    assert fl["nout"] == 512 and fl["kernel"] == "one CTA per tile"
     for part in (fl, fl["backward"]):
         r = part["roofline"]
         assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and 0 < r["frac"] < 1.5
