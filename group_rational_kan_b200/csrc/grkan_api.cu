@@ -694,20 +694,16 @@ void quad_cols(int64_t nout, int* np, int* n_ct) {
   *np = (int)((share + 127) / 128 * 128);
 }
 
-// Whether grkan_linear_forward takes the cluster kernel. Its K steps cost about
-// the same time whatever the tile width (the activation path, not the tensor
-// cores, sets the pace), so it pays where a cluster's column tile is wide: one
-// tile of more than 512 outputs, or tiles whose pairs are 512 wide. Measured on
-// the KAT-B rows (100,864 x 3072): n_out 576 to 1024, 2048 and (d 768) 3072 are
-// faster than the one-CTA kernel; 512 and below, and 1536 (two tiles of 768),
-// are slower.
+// Whether grkan_linear_forward takes the cluster kernel: for n_out > 512 (d a
+// multiple of its K step). Measured on the KAT-B rows (100,864 x 3072): n_out 576
+// to 2048 are faster than or level with the one-CTA kernel (768: 0.53 against
+// 0.68 ms; 1536, two column tiles of 768: 1.02 against 1.06), and at d = 768
+// n_out 1536 and 3072 are 24-37 % faster; n_out 512 and below are slower (512:
+// 0.50 against 0.41), where the one-CTA kernel already activates each element
+// once.
 bool use_linear_quad(const Plan& p, int64_t nout) {
   if (!GRK_LIN_QUAD || p.d % grk::lin::qd::BK != 0) return false;
-  if (GRK_LIN_QUAD == 2) return true;
-  if (nout <= 512) return false;
-  int np = 0, n_ct = 0;
-  quad_cols(nout, &np, &n_ct);
-  return n_ct == 1 || np == grk::lin::qd::kNPMax;
+  return GRK_LIN_QUAD == 2 || nout > 512;
 }
 
 // The cluster fused forward: d a multiple of its K step (64); the plan, the

@@ -48,9 +48,8 @@
 
 #include "grkan_linear_bwd.cuh"
 
-// 1: grkan_linear_forward takes this kernel for the shapes where it is the
-// faster of the two (use_linear_quad in grkan_api.cu); 2: whenever d is a
-// multiple of 64; 0: never.
+// 1: grkan_linear_forward takes this kernel for n_out > 512 (use_linear_quad in
+// grkan_api.cu); 2: whenever d is a multiple of 64; 0: never.
 #ifndef GRK_LIN_QUAD
 #define GRK_LIN_QUAD 1
 #endif

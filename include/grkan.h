@@ -158,11 +158,10 @@ GRKAN_API grkan_status_t grkan_linear_forward(const void* x, const float* a, con
                                               grkan_dtype_t dtype, void* stream);
 
 /* Which kernel grkan_linear_forward takes for these shapes: 1 = clusters of four
- * CTAs (two tcgen05 CTA pairs sharing each 256-row tile; n_out > 512 when one
- * column tile, or 512-wide pairs, cover the outputs, and d % 64 == 0), 0 = one
- * CTA per 128 x 512 output tile, < 0 = the negated status the call would return
- * for these shapes. Both kernels give the same bits. No device is queried: on a
- * device where no cluster of four fits, a 1 runs as 0. */
+ * CTAs (two tcgen05 CTA pairs sharing each 256-row tile; n_out > 512 and
+ * d % 64 == 0), 0 = one CTA per 128 x 512 output tile, < 0 = the negated status
+ * the call would return for these shapes. Both kernels give the same bits. No
+ * device is queried: on a device where no cluster of four fits, a 1 runs as 0. */
 GRKAN_API int32_t grkan_linear_forward_path(int64_t B, int64_t N, int64_t d, int32_t n_g,
                                             int32_t m, int32_t n, int64_t nout,
                                             grkan_dtype_t dtype);

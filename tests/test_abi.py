@@ -72,8 +72,8 @@ def test_path_selection():
 
 def test_linear_forward_path():
     """The fused linear forward's kernel by shape (no device needed): the cluster
-    kernel for n_out > 512 when one column tile or 512-wide pairs cover it and d is
-    a multiple of 64, the one-CTA kernel otherwise."""
+    kernel for n_out > 512 when d is a multiple of 64, the one-CTA kernel
+    otherwise."""
     p = grk.grkan_linear_forward_path
     kat_b = (512, 197, 3072, 8, 5, 4)
     assert p(*kat_b, 768, grk.BF16) == 1    # one tile, pairs of 384
@@ -81,7 +81,8 @@ def test_linear_forward_path():
     assert p(*kat_b, 576, grk.BF16) == 1
     assert p(*kat_b, 512, grk.BF16) == 0    # one 512-column pass of the one-CTA kernel
     assert p(*kat_b, 384, grk.BF16) == 0
-    assert p(*kat_b, 1536, grk.BF16) == 0   # two tiles with pairs of 384
+    assert p(*kat_b, 1536, grk.BF16) == 1   # two tiles with pairs of 384
+    assert p(*kat_b, 520, grk.BF16) == 1    # just past one 512-column pass
     assert p(*kat_b, 2048, grk.BF16) == 1   # two tiles with pairs of 512
     assert p(512, 197, 768, 8, 5, 4, 3072, grk.BF16) == 1   # three tiles of 1024
     assert p(2, 3, 160, 20, 5, 4, 768, grk.BF16) == 0       # d not a multiple of 64
